@@ -1,0 +1,166 @@
+"""Plain fp64 CPU oracle for RoPE + grouped-query causal scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports, calls or links this
+module: only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it. It shares no code with the CUDA
+library; both sides receive the same seeded inputs from ``synthetic``.
+
+Everything is written the slow, obvious way: numpy float64, the full score block
+materialised per (batch, head), an explicit -inf mask, a plain row softmax. The
+functions follow these passages:
+
+* "Multi-Head Attention & Rotary Position Embeddings (RoPE)" (learnllm.online),
+  section "Scaled Dot-Product Attention: The O(S^2) Memory Wall" and its
+  ``scaled_dot_product_attention`` code: scores = Q K^T / sqrt(d_k), an upper
+  triangle of -inf above the diagonal when causal, softmax over the last axis,
+  weights times V.
+* "Transformer Architecture & Self-Attention Mechanics" (devthesis.com), §1
+  (the row-wise softmax A_ij = exp(q_i.k_j/sqrt d_k) / sum_l exp(q_i.k_l/sqrt d_k))
+  and §3 "Rotary Position Embeddings (RoPE)": pairs (q_2i, q_2i+1) rotated by
+  R(m theta_i) = [[cos, -sin], [sin, cos]], theta_i = 10000^(-2i/d_k).
+* "Transformer internals: attention without the mysticism" (ninaddeshpande.com),
+  section "Rotary positional embeddings (RoPE)": the base b of theta_i is a free
+  parameter (context extension changes it), and section "The KV cache and the
+  memory wall": grouped-query attention shares one key/value head among a group
+  of query heads.
+* "Building Self-Attention and Transformer Engines" (codingpancake.com), FAQ Q2:
+  causal masking sets the upper triangle to -inf before the softmax.
+
+Readings where the pages leave a step open (each also listed in the design notes):
+
+* Head sharing: query head h reads key/value head h // (Hq // Hkv) (contiguous
+  groups), Hq a multiple of Hkv.
+* Positions are bottom-right aligned: query row i sits at absolute position
+  pos_offset + (Sk - Sq) + i, key row j at pos_offset + j, and key j is allowed
+  iff its position is not after the query's. At Sq == Sk and pos_offset == 0 this
+  is exactly triu(-inf, diagonal=1).
+* Pairs are adjacent elements (2i, 2i+1); theta_i = base^(-2i/D), i = 0..D/2-1;
+  every one of the D dimensions is rotated.
+* Decode: the single query at absolute position ``pos`` attends cache rows
+  0..min(Sk, pos+1)-1, which hold keys that were already rotated when written.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "rope_inv_freq",
+    "rope_rotate",
+    "attention",
+    "query_positions",
+    "rope_attn_fwd",
+    "rope_attn_decode",
+]
+
+
+def rope_inv_freq(D: int, base: float) -> np.ndarray:
+    """theta_i = base^(-2i/D) for i = 0..D/2-1 (devthesis §3 RoPE; base b per
+    ninaddeshpande "Rotary positional embeddings")."""
+    if D % 2:
+        raise ValueError("RoPE needs an even head dimension")
+    i = np.arange(D // 2, dtype=np.float64)
+    return np.power(np.float64(base), -2.0 * i / D)
+
+
+def rope_rotate(x: np.ndarray, positions: np.ndarray, base: float) -> np.ndarray:
+    """Rotate every adjacent pair (x_2i, x_2i+1) of the rows of ``x`` by m*theta_i.
+
+    ``x`` has shape [..., S, D]; ``positions`` holds the S absolute positions m.
+    Per pair: x'_2i = x_2i cos - x_2i+1 sin, x'_2i+1 = x_2i sin + x_2i+1 cos, the
+    matrix R(m theta_i) of devthesis §3 applied to the column (x_2i, x_2i+1).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    theta = rope_inv_freq(D, base)                                   # [D/2]
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * theta[None, :]  # [S, D/2]
+    c, s = np.cos(ang), np.sin(ang)
+    even, odd = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = even * c - odd * s
+    out[..., 1::2] = even * s + odd * c
+    return out
+
+
+def query_positions(Sq: int, Sk: int, pos_offset: int) -> np.ndarray:
+    """Absolute positions of the Sq query rows (bottom-right aligned with the keys)."""
+    return pos_offset + (Sk - Sq) + np.arange(Sq, dtype=np.int64)
+
+
+def _softmax_rows(s: np.ndarray) -> np.ndarray:
+    """Row softmax: subtract the row max, exponentiate, divide by the row sum."""
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool,
+              rows: np.ndarray | None = None, row_block: int = 1024) -> np.ndarray:
+    """softmax(Q K^T / sqrt(D) + M) V with grouped KV heads, in float64.
+
+    q: [B, Hq, Sq, D]; k, v: [B, Hkv, Sk, D] (no RoPE applied here).
+    M is -inf where key j lies after query i under the bottom-right alignment
+    (j > i + Sk - Sq), i.e. numpy's triu with offset Sk - Sq + 1; zero elsewhere.
+    ``rows`` optionally selects which query rows to compute (each row of attention
+    is independent of the others, so a subset is an exact check of those rows).
+    The score block is materialised ``row_block`` rows at a time to bound memory.
+    Returns float64 [B, Hq, len(rows) or Sq, D].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Sk, _ = k.shape
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    rows = np.arange(Sq) if rows is None else np.asarray(rows, dtype=np.int64)
+    scale = 1.0 / np.sqrt(np.float64(D))
+    out = np.empty((B, Hq, rows.size, v.shape[-1]), dtype=np.float64)
+    cols = np.arange(Sk)
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // G
+            for r0 in range(0, rows.size, row_block):
+                r = rows[r0:r0 + row_block]
+                s = (q[b, h, r] @ k[b, kv].T) * scale            # [R, Sk]
+                if causal:
+                    s = np.where(cols[None, :] > (r[:, None] + (Sk - Sq)), -np.inf, s)
+                out[b, h, r0:r0 + r.size] = _softmax_rows(s) @ v[b, kv]
+    return out
+
+
+def rope_attn_fwd(q, k, v, rope_base: float, pos_offset: int = 0, causal: bool = True,
+                  rows=None) -> np.ndarray:
+    """The prefill result: rotate Q and K by their absolute positions, then attend.
+
+    q: [B, Hq, Sq, D]; k, v: [B, Hkv, Sk, D]; inputs are widened to float64 first.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    Sq, Sk = q.shape[2], k.shape[2]
+    qpos = query_positions(Sq, Sk, pos_offset)
+    kpos = pos_offset + np.arange(Sk, dtype=np.int64)
+    if rows is not None:
+        # rotating only the selected query rows is the same arithmetic per row
+        rows = np.asarray(rows, dtype=np.int64)
+        q_sel = np.zeros_like(q)
+        q_sel[:, :, rows] = rope_rotate(q[:, :, rows], qpos[rows], rope_base)
+        q_rot = q_sel
+    else:
+        q_rot = rope_rotate(q, qpos, rope_base)
+    k_rot = rope_rotate(k, kpos, rope_base)
+    return attention(q_rot, k_rot, v, causal, rows=rows)
+
+
+def rope_attn_decode(q, k_cache_rot, v_cache, rope_base: float, pos: int) -> np.ndarray:
+    """One decode step: the query at absolute position ``pos`` (rotated here) attends
+    the first min(Sk, pos+1) rows of an already-rotated key cache.
+
+    q: [B, Hq, 1, D]; k_cache_rot, v_cache: [B, Hkv, Sk, D]. Returns [B, Hq, 1, D].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Sk = k_cache_rot.shape[2]
+    L = min(Sk, pos + 1)
+    q_rot = rope_rotate(q, np.array([pos]), rope_base)
+    return attention(q_rot, np.asarray(k_cache_rot)[:, :, :L], np.asarray(v_cache)[:, :, :L],
+                     causal=False)

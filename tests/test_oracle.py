@@ -1,0 +1,330 @@
+"""Pins for the fp64 oracle: values the pages print, closed forms, invariants, an
+independent brute force and a library cross-check. CPU only.
+
+Each test targets a plausible mistake in the oracle (a wrong rotation sense, a
+dropped 1/sqrt(D), a transposed operand, an off-by-one in the mask, a wrong head
+map); ``test_planted_mistakes_are_caught`` plants such mistakes in a copy of the
+oracle and checks that a pin fails for each.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import read_golden
+import oracle
+from oracle import ref
+from synthetic import TINY, Workload, make_inputs, to_f64
+
+
+# ----------------------------------------------------------------- pages' values
+
+def _weights_of_one_query(logits, d_k):
+    """Attention weights of one query over len(logits) keys whose raw dot products
+    with it are ``logits``: q = (c, 0, ...), key_j = (logit_j / c, 0, ...), V = identity."""
+    n = len(logits)
+    c = 4.0
+    q = np.zeros((1, 1, 1, d_k))
+    q[0, 0, 0, 0] = c
+    k = np.zeros((1, 1, n, d_k))
+    k[0, 0, :, 0] = np.asarray(logits) / c
+    v = np.zeros((1, 1, n, n))
+    v[0, 0] = np.eye(n)
+    return oracle.attention(q, k, v, causal=False)[0, 0, 0]
+
+
+def test_problem1_scaled_softmax_weights():
+    g = read_golden("problem1_scaled_softmax.txt")
+    w = _weights_of_one_query(g["logits"], int(g["d_k"]))
+    np.testing.assert_allclose(w, g["scaled_weights"], atol=g["scaled_weights_tol"], rtol=0)
+
+
+def test_problem1_unscaled_is_not_what_oracle_computes():
+    # with d_k = 1 the 1/sqrt(d_k) factor is 1, which reproduces the page's unscaled row;
+    # at d_k = 64 the oracle must NOT give it (pins that the scale is applied).
+    g = read_golden("problem1_scaled_softmax.txt")
+    w1 = _weights_of_one_query(g["logits"], 1)
+    np.testing.assert_allclose(w1, g["unscaled_weights"], atol=g["unscaled_weights_tol"], rtol=0)
+    w64 = _weights_of_one_query(g["logits"], 64)
+    assert abs(w64[0] - g["unscaled_weights"][0]) > 0.3
+
+
+def test_problem2_two_token_head():
+    g = read_golden("problem2_head_output.txt")
+    Q = np.array(g["Q1"])[None, None]
+    K = np.array(g["K1"])[None, None]
+    V = np.array(g["V1"])[None, None]
+    H = oracle.attention(Q, K, V, causal=False)[0, 0]
+    np.testing.assert_allclose(H, np.array(g["H1"]), atol=g["tol"], rtol=0)
+    # the weights themselves: V = I returns A
+    A = oracle.attention(Q, K, np.eye(2)[None, None], causal=False)[0, 0]
+    np.testing.assert_allclose(A, np.array(g["A1"]), atol=g["tol"], rtol=0)
+
+
+def test_problem3_rope_sign_pin():
+    g = read_golden("problem3_rope_relative.txt")
+    q = np.array(g["q"])[None, :]
+    k = np.array(g["k"])[None, :]
+    qr = oracle.rope_rotate(q, np.array([int(g["m"])]), 10000.0)
+    kr = oracle.rope_rotate(k, np.array([int(g["n"])]), 10000.0)
+    assert abs(float(qr[0] @ kr[0]) - g["value"]) < g["tol"]
+
+
+@pytest.mark.parametrize("D,base", [(2, 10000.0), (8, 10000.0), (64, 10000.0), (128, 500000.0)])
+def test_problem3_rope_closed_form_random(D, base):
+    rng = np.random.default_rng(1)
+    theta = base ** (-2.0 * np.arange(D // 2) / D)
+    for _ in range(20):
+        q, k = rng.standard_normal(D), rng.standard_normal(D)
+        m, n = rng.integers(0, 40000, size=2)
+        qr = oracle.rope_rotate(q[None], np.array([m]), base)[0]
+        kr = oracle.rope_rotate(k[None], np.array([n]), base)[0]
+        for i in range(D // 2):
+            q1, q2, k1, k2 = q[2 * i], q[2 * i + 1], k[2 * i], k[2 * i + 1]
+            dot, cross = q1 * k1 + q2 * k2, q2 * k1 - q1 * k2
+            want = dot * math.cos((m - n) * theta[i]) - cross * math.sin((m - n) * theta[i])
+            got = qr[2 * i] * kr[2 * i] + qr[2 * i + 1] * kr[2 * i + 1]
+            assert abs(got - want) < 1e-9 * (1 + abs(dot) + abs(cross))
+
+
+# ----------------------------------------------------------------- RoPE properties
+
+def test_rope_position_zero_is_identity():
+    # the page-5 demo rotates a token at position 0: R_0 = I
+    x = np.random.default_rng(2).standard_normal((5, 64))
+    np.testing.assert_array_equal(oracle.rope_rotate(x, np.zeros(5, dtype=np.int64), 10000.0), x)
+
+
+@pytest.mark.parametrize("D,base", [(8, 10000.0), (64, 10000.0), (128, 500000.0)])
+def test_rope_frequencies(D, base):
+    # pair i of a unit vector along x_2i, at position 1, turns by exactly base^(-2i/D)
+    x = np.zeros((D // 2, D))
+    for i in range(D // 2):
+        x[i, 2 * i] = 1.0
+    r = oracle.rope_rotate(x, np.ones(D // 2, dtype=np.int64), base)
+    for i in range(D // 2):
+        ang = math.atan2(r[i, 2 * i + 1], r[i, 2 * i])
+        assert abs(ang - base ** (-2.0 * i / D)) < 1e-14
+
+
+def test_rope_is_complex_multiplication():
+    # independent formulation: pair (x_2i, x_2i+1) as z = x_2i + i x_2i+1, times e^{i m theta}
+    rng = np.random.default_rng(3)
+    D, base = 64, 10000.0
+    x = rng.standard_normal((7, D))
+    pos = rng.integers(0, 100000, size=7)
+    z = x[:, 0::2] + 1j * x[:, 1::2]
+    theta = np.array([base ** (-2.0 * i / D) for i in range(D // 2)])
+    zr = z * np.exp(1j * pos[:, None] * theta[None, :])
+    r = oracle.rope_rotate(x, pos, base)
+    np.testing.assert_allclose(r[:, 0::2], zr.real, atol=1e-9)
+    np.testing.assert_allclose(r[:, 1::2], zr.imag, atol=1e-9)
+    # rotations keep norms
+    np.testing.assert_allclose(np.linalg.norm(r, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+
+
+def test_relative_invariance_through_pos_offset():
+    q, k, v = (to_f64(t) for t in make_inputs(Workload("t", 1, 2, 2, 48, 48, 16, 10000.0), seed=4))
+    o0 = oracle.rope_attn_fwd(q, k, v, 10000.0, pos_offset=0)
+    for c in (1, 17, 12345):
+        oc = oracle.rope_attn_fwd(q, k, v, 10000.0, pos_offset=c)
+        np.testing.assert_allclose(oc, o0, atol=1e-10, rtol=0)
+
+
+# ----------------------------------------------------------------- attention invariants
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def test_rows_sum_to_one():
+    q, k = _rand((2, 4, 33, 16), 5), _rand((2, 2, 33, 16), 6)
+    v = np.ones((2, 2, 33, 16))
+    for causal in (True, False):
+        o = oracle.rope_attn_fwd(q, k, v, 10000.0, causal=causal)
+        np.testing.assert_allclose(o, 1.0, atol=1e-13)
+
+
+def test_causal_row0_is_v0():
+    q, k, v = _rand((1, 3, 40, 16), 7), _rand((1, 3, 40, 16), 8), _rand((1, 3, 40, 16), 9)
+    o = oracle.rope_attn_fwd(q, k, v, 10000.0, causal=True)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0], atol=1e-14, rtol=0)
+
+
+def test_zero_q_gives_prefix_mean():
+    S = 50
+    q = np.zeros((1, 2, S, 16))
+    k, v = _rand((1, 2, S, 16), 10), _rand((1, 2, S, 16), 11)
+    o = oracle.rope_attn_fwd(q, k, v, 10000.0, causal=True)
+    prefix = np.cumsum(v, axis=2) / np.arange(1, S + 1)[None, None, :, None]
+    np.testing.assert_allclose(o, prefix, atol=1e-13)
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    q, k, v = _rand((2, 8, 30, 16), 12), _rand((2, 2, 30, 16), 13), _rand((2, 2, 30, 16), 14)
+    o = oracle.rope_attn_fwd(q, k, v, 10000.0)
+    o_mha = oracle.rope_attn_fwd(q, np.repeat(k, 4, axis=1), np.repeat(v, 4, axis=1), 10000.0)
+    np.testing.assert_allclose(o, o_mha, atol=1e-13, rtol=0)
+    # and the head map is contiguous: head 5 reads kv head 1, not kv head 5 % 2
+    o_wrong = oracle.rope_attn_fwd(q, np.tile(k, (1, 4, 1, 1)), np.tile(v, (1, 4, 1, 1)), 10000.0)
+    assert np.max(np.abs(o_wrong[:, 1] - o[:, 1])) > 1e-3
+
+
+def test_permutation_equivariance():
+    # without mask and rotation, attention(P X) = P attention(X): permuting keys and values
+    # together leaves the output alone; permuting queries permutes the output
+    q, k, v = _rand((1, 1, 12, 8), 15), _rand((1, 1, 12, 8), 16), _rand((1, 1, 12, 8), 17)
+    p = np.random.default_rng(18).permutation(12)
+    o = oracle.attention(q, k, v, causal=False)
+    np.testing.assert_allclose(oracle.attention(q, k[:, :, p], v[:, :, p], causal=False), o, atol=1e-13)
+    np.testing.assert_allclose(oracle.attention(q[:, :, p], k, v, causal=False), o[:, :, p], atol=1e-13)
+
+
+def test_score_variance_is_one():
+    # iid N(0,1) rotated q, k: q.k / sqrt(D) has mean 0 and variance 1 (devthesis §1)
+    q, k, _ = (to_f64(t) for t in make_inputs(Workload("s", 1, 1, 1, 2048, 2048, 128, 500000.0), seed=19))
+    pos = np.arange(2048)
+    qr = oracle.rope_rotate(q[0, 0], pos, 500000.0)
+    kr = oracle.rope_rotate(k[0, 0], pos, 500000.0)
+    s = (qr @ kr.T).ravel() / math.sqrt(128)
+    assert abs(s.mean()) < 0.01 and abs(s.var() - 1.0) < 0.02
+
+
+def test_bottom_right_alignment():
+    # Sq < Sk: the last Sq rows of the full Sq == Sk problem, with the same positions
+    q, k, v = _rand((1, 2, 40, 16), 20), _rand((1, 2, 40, 16), 21), _rand((1, 2, 40, 16), 22)
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0, pos_offset=3)
+    part = oracle.rope_attn_fwd(q[:, :, 25:], k, v, 10000.0, pos_offset=3)
+    np.testing.assert_allclose(part, full[:, :, 25:], atol=1e-13, rtol=0)
+
+
+def test_rows_subset_matches_full():
+    q, k, v = _rand((1, 2, 70, 16), 23), _rand((1, 1, 70, 16), 24), _rand((1, 1, 70, 16), 25)
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0)
+    rows = np.array([0, 5, 31, 69])
+    np.testing.assert_allclose(oracle.rope_attn_fwd(q, k, v, 10000.0, rows=rows),
+                               full[:, :, rows], atol=1e-14, rtol=0)
+
+
+def test_decode_equals_last_prefill_row():
+    S = 37
+    q, k, v = _rand((2, 4, S, 16), 26), _rand((2, 2, S, 16), 27), _rand((2, 2, S, 16), 28)
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0)
+    k_cache = oracle.rope_rotate(k, np.arange(S), 10000.0)
+    d = oracle.rope_attn_decode(q[:, :, S - 1:], k_cache, v, 10000.0, pos=S - 1)
+    np.testing.assert_allclose(d[:, :, 0], full[:, :, S - 1], atol=1e-13, rtol=0)
+    # a longer cache with rows past pos is ignored
+    pad = np.concatenate([k_cache, _rand((2, 2, 5, 16), 29)], axis=2)
+    vpad = np.concatenate([v, _rand((2, 2, 5, 16), 30)], axis=2)
+    d2 = oracle.rope_attn_decode(q[:, :, S - 1:], pad, vpad, 10000.0, pos=S - 1)
+    np.testing.assert_allclose(d2, d, atol=1e-15, rtol=0)
+
+
+# ----------------------------------------------------------------- independent brute force
+
+def _brute(q, k, v, base, pos_offset, causal):
+    """Scalar loops, math.fsum and math.cos/sin; written separately from the oracle."""
+    B, Hq, Sq, D = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv, Sk = len(k[0]), len(k[0][0])
+
+    def rot(vec, p):
+        out = [0.0] * D
+        for i in range(D // 2):
+            a = p * base ** (-2.0 * i / D)
+            c, s = math.cos(a), math.sin(a)
+            out[2 * i] = vec[2 * i] * c - vec[2 * i + 1] * s
+            out[2 * i + 1] = vec[2 * i] * s + vec[2 * i + 1] * c
+        return out
+
+    res = []
+    for b in range(B):
+        hb = []
+        for h in range(Hq):
+            g = h * Hkv // Hq
+            rows = []
+            for i in range(Sq):
+                pi = pos_offset + Sk - Sq + i
+                qi = rot(q[b][h][i], pi)
+                sc = []
+                for j in range(Sk):
+                    pj = pos_offset + j
+                    if causal and pj > pi:
+                        continue
+                    kj = rot(k[b][g][j], pj)
+                    sc.append((j, math.fsum(x * y for x, y in zip(qi, kj)) / math.sqrt(D)))
+                mx = max(s for _, s in sc)
+                w = [(j, math.exp(s - mx)) for j, s in sc]
+                z = math.fsum(e for _, e in w)
+                rows.append([math.fsum(e * v[b][g][j][d] for j, e in w) / z for d in range(D)])
+            hb.append(rows)
+        res.append(hb)
+    return np.array(res)
+
+
+@pytest.mark.parametrize("Sq,Sk,causal,off", [(8, 8, True, 0), (5, 8, True, 3), (8, 8, False, 0),
+                                              (1, 6, True, 9), (7, 3, False, 2)])
+def test_brute_force_small(Sq, Sk, causal, off):
+    rng = np.random.default_rng(31)
+    q = rng.standard_normal((1, 4, Sq, 6))
+    k = rng.standard_normal((1, 2, Sk, 6))
+    v = rng.standard_normal((1, 2, Sk, 6))
+    want = _brute(q.tolist(), k.tolist(), v.tolist(), 10000.0, off, causal)
+    got = oracle.rope_attn_fwd(q, k, v, 10000.0, pos_offset=off, causal=causal)
+    np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
+
+
+def test_torch_sdpa_crosscheck():
+    # library cross-check: torch's CPU fp64 SDPA on independently rotated Q/K (complex form)
+    q, k, v = (to_f64(t) for t in make_inputs(TINY, seed=0))
+    D, S, base = TINY.D, TINY.Sq, TINY.rope_base
+    theta = np.array([base ** (-2.0 * i / D) for i in range(D // 2)])
+    rot = lambda x: (lambda z: np.stack([z.real, z.imag], -1).reshape(x.shape))(
+        (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * np.arange(S)[:, None] * theta))
+    qt, kt, vt = (torch.from_numpy(a) for a in (rot(q), rot(k), v))
+    want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True).numpy()
+    got = oracle.rope_attn_fwd(q, k, v, base)
+    np.testing.assert_allclose(got, want, atol=1e-10, rtol=0)
+
+
+# ----------------------------------------------------------------- planted mistakes
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Plant typical mistakes in the oracle (CPU) and check that some pin fails."""
+    g3 = read_golden("problem3_rope_relative.txt")
+
+    def sign_pin():
+        qr = ref.rope_rotate(np.array([[1.0, 0.0]]), np.array([1]), 10000.0)
+        kr = ref.rope_rotate(np.array([[0.0, 1.0]]), np.array([0]), 10000.0)
+        return abs(float(qr[0] @ kr[0]) - g3["value"]) < g3["tol"]
+
+    def problem1_pin():
+        g = read_golden("problem1_scaled_softmax.txt")
+        return np.allclose(_weights_of_one_query(g["logits"], 64), g["scaled_weights"], atol=1e-5)
+
+    def causal_pin():
+        q, k, v = _rand((1, 1, 9, 4), 40), _rand((1, 1, 9, 4), 41), _rand((1, 1, 9, 4), 42)
+        o = ref.rope_attn_fwd(q, k, v, 10000.0)
+        return np.allclose(o[:, :, 0], v[:, :, 0], atol=1e-14)
+
+    assert sign_pin() and problem1_pin() and causal_pin()
+
+    orig_rot = ref.rope_rotate
+
+    def wrong_sense(x, positions, base):
+        return orig_rot(x, -np.asarray(positions), base)
+    monkeypatch.setattr(ref, "rope_rotate", wrong_sense)
+    assert not sign_pin()
+    monkeypatch.setattr(ref, "rope_rotate", orig_rot)
+
+    orig_sm = ref._softmax_rows
+    monkeypatch.setattr(ref, "_softmax_rows", lambda s: orig_sm(s * math.sqrt(64)))  # scale dropped
+    assert not problem1_pin()
+    monkeypatch.setattr(ref, "_softmax_rows", orig_sm)
+
+    orig_attn = ref.attention
+
+    def no_mask(q, k, v, causal, rows=None, row_block=1024):
+        return orig_attn(q, k, v, False, rows, row_block)
+    monkeypatch.setattr(ref, "attention", no_mask)
+    assert not causal_pin()
