@@ -1,0 +1,133 @@
+/*
+ * libropeattn: exact causal scaled-dot-product attention with RoPE and grouped-query
+ * key/value sharing, for NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every tensor argument is a plain pointer to caller-owned DEVICE memory holding
+ * bf16 values (IEEE bfloat16, 2 bytes) in contiguous BHSD layout
+ * [batch][heads][seq][head_dim], head_dim innermost. Pointers must be 16-byte aligned;
+ * outputs must not overlap inputs. All calls are asynchronous with respect to the host:
+ * they validate the arguments, enqueue work on `stream` (NULL = legacy default stream)
+ * and return. A non-RA_OK return means nothing was enqueued (argument errors) or a CUDA
+ * launch/allocation failed (RA_ERR_CUDA). Errors found by the kernels themselves (a wait
+ * that ran out) are sticky and read with rope_attn_get_device_status().
+ *
+ * The positions follow the bottom-right alignment used throughout: query row i sits at
+ * absolute position pos_offset + (Sk - Sq) + i, key row j at pos_offset + j, and under the
+ * causal mask key j is visible to query i iff its position is not after the query's.
+ *
+ * Temporary device memory (the rotated keys and the RoPE table of rope_attn_fwd, the
+ * per-split partials of rope_attn_decode) is taken with cudaMallocAsync on `stream` and
+ * released with cudaFreeAsync on the same stream before the call returns.
+ */
+#ifndef ROPEATTN_H_
+#define ROPEATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RA_API __attribute__((visibility("default")))
+#else
+#define RA_API
+#endif
+
+struct CUstream_st; /* the same handle type as cudaStream_t / CUstream */
+typedef struct CUstream_st* ra_stream_t;
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad size, aliasing, Hq % Hkv != 0 ... */
+  RA_ERR_UNSUPPORTED = 2,    /* valid request outside what the kernels implement (D not 64/128) */
+  RA_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed; see rope_attn_last_cuda_error */
+  RA_ERR_DEVICE_TIMEOUT = 4  /* a kernel gave up waiting on one of its own barriers */
+} ra_status;
+
+/*
+ * Prefill / full-sequence attention.
+ *
+ *   out[b,h,i,:] = sum_j softmax_j( <R(p_q(i)) q[b,h,i,:], R(p_k(j)) k[b,h/G,j,:]> / sqrt(D) + M_ij )
+ *                  * v[b,h/G,j,:]
+ *
+ * Scaled dot-product attention softmax(QK^T/sqrt(d_k))V as defined in "Transformer
+ * Architecture & Self-Attention Mechanics" (devthesis.com), §1, with the causal -inf upper
+ * triangle of "Multi-Head Attention & Rotary Position Embeddings (RoPE)" (learnllm.online,
+ * its scaled_dot_product_attention code), the rotary embedding of devthesis §3 "Rotary
+ * Position Embeddings (RoPE)" (pairs (x_2i, x_2i+1) turned by m*base^(-2i/D)), and the
+ * grouped-query sharing of "Transformer internals: attention without the mysticism"
+ * (ninaddeshpande.com, "The KV cache and the memory wall"): G = Hq/Hkv query heads share
+ * one key/value head, query head h reading kv head h / G.
+ *
+ *   q    [B, Hq,  Sq, D] bf16 (read)          k, v [B, Hkv, Sk, D] bf16 (read)
+ *   out  [B, Hq,  Sq, D] bf16 (written)
+ *   D in {64, 128}; Hq % Hkv == 0; all sizes >= 1; causal requires Sq <= Sk.
+ *   rope_base > 0 and finite; pos_offset >= 0 (absolute position of key row 0).
+ *   causal: nonzero = apply the causal mask; zero = attend all Sk keys.
+ * Returns RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED or RA_ERR_CUDA.
+ */
+RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                        int Hkv, int Sq, int Sk, int D, float rope_base, int pos_offset,
+                        int causal, ra_stream_t stream);
+
+/*
+ * RoPE rotation of a whole tensor (builds a pre-rotated key cache for rope_attn_decode).
+ *
+ *   x_rot[b,h,s,2i]   = x[b,h,s,2i] cos(m theta_i) - x[b,h,s,2i+1] sin(m theta_i)
+ *   x_rot[b,h,s,2i+1] = x[b,h,s,2i] sin(m theta_i) + x[b,h,s,2i+1] cos(m theta_i)
+ *   m = pos_offset + s, theta_i = rope_base^(-2i/D)
+ *
+ * devthesis.com §3 "Rotary Position Embeddings (RoPE)"; the base is a parameter as in
+ * ninaddeshpande.com "Rotary positional embeddings (RoPE)".
+ *   x, x_rot [B, H, S, D] bf16; x_rot may equal x (in place) but not overlap it otherwise.
+ *   D even, 8 <= D <= 256 and D % 8 == 0; pos_offset >= 0. Angles are formed in fp64.
+ */
+RA_API ra_status rope_attn_rotate(const void* x, void* x_rot, int B, int H, int S, int D,
+                           float rope_base, int pos_offset, ra_stream_t stream);
+
+/*
+ * One decode step over a pre-rotated KV cache (split-KV with a log-sum-exp combine).
+ *
+ * The query of each head, at absolute position `pos`, is rotated by R(pos) and attends
+ * cache rows j = 0 .. L-1, L = min(Sk, pos + 1), which hold keys already rotated to their
+ * own positions (as written by rope_attn_rotate) and their values:
+ *   out[b,h,0,:] = sum_{j<L} softmax_j(<R(pos) q[b,h,0,:], k_cache_rot[b,h/G,j,:]> / sqrt(D))
+ *                  * v_cache[b,h/G,j,:]
+ * ("Transformer internals: attention without the mysticism", "The KV cache and the memory
+ * wall": decoding keeps the past keys and values and reads all of them every step.)
+ *   q [B, Hq, 1, D] bf16; k_cache_rot, v_cache [B, Hkv, Sk, D] bf16; out [B, Hq, 1, D].
+ *   D in {64, 128}; Hq % Hkv == 0; pos >= 0; n_splits = 0 picks the split count, otherwise
+ *   the number of key ranges (clamped to what L allows).
+ */
+RA_API ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const void* v_cache,
+                           void* out, int B, int Hq, int Hkv, int Sk, int D, float rope_base,
+                           int pos, int n_splits, ra_stream_t stream);
+
+/* Split count rope_attn_decode uses for these sizes when n_splits == 0. */
+RA_API int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos);
+
+/*
+ * Synchronises `stream`, returns the sticky device status of the current device
+ * (RA_OK or RA_ERR_DEVICE_TIMEOUT) and clears it; RA_ERR_CUDA if the sync itself failed.
+ */
+RA_API ra_status rope_attn_get_device_status(ra_stream_t stream);
+
+/*
+ * Polls each kernel wait makes before it gives up and reports RA_ERR_DEVICE_TIMEOUT
+ * (default 1<<26). A test knob: 0 makes every wait give up at once, without polling, so the
+ * timeout path runs while the kernels still exit cleanly. Returns the previous value;
+ * limit < 0 only queries.
+ */
+RA_API long long rope_attn_set_wait_limit(long long limit);
+
+/* Text of a status code; the last CUDA error string for RA_ERR_CUDA. */
+RA_API const char* rope_attn_status_string(int status);
+RA_API const char* rope_attn_last_cuda_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+RA_API int rope_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROPEATTN_H_ */

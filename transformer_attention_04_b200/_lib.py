@@ -1,0 +1,148 @@
+"""ctypes binding of libropeattn (include/ropeattn.h).
+
+Argument marshalling only: tensors are checked for device, dtype, layout and shape,
+and their data pointers plus the current CUDA stream are passed to the C ABI. Every
+step of the computation runs in the library's CUDA kernels; there is no fallback,
+and a missing library raises at first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libropeattn.so")
+
+RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_DEVICE_TIMEOUT = range(5)
+
+# name -> (restype, argtypes), exactly the functions include/ropeattn.h declares
+_P, _I, _F, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+SIGNATURES = {
+    "rope_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "rope_attn_rotate": (_I, [_P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "rope_attn_decode": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "rope_attn_decode_auto_splits": (_I, [_I, _I, _I, _I, _I, _I]),
+    "rope_attn_get_device_status": (_I, [_P]),
+    "rope_attn_set_wait_limit": (_LL, [_LL]),
+    "rope_attn_status_string": (ctypes.c_char_p, [_I]),
+    "rope_attn_last_cuda_error": (ctypes.c_char_p, []),
+    "rope_attn_version": (_I, []),
+}
+
+_lib = None
+
+
+class RopeAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lib().rope_attn_status_string(status).decode()
+        super().__init__(f"{where}: status {status} ({msg})")
+        self.status = status
+
+
+def lib():
+    """Load libropeattn.so (built in-tree by transformer_attention_04_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m transformer_attention_04_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = handle
+    return _lib
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(t: torch.Tensor, name: str, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (BHSD)")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _raise(status, where):
+    if status != RA_OK:
+        raise RopeAttnError(status, where)
+
+
+def rope_attn_fwd(q, k, v, rope_base: float, pos_offset: int = 0, causal: bool = True,
+                  out=None, stream=None):
+    """Prefill attention. q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D] bf16 CUDA; returns out [B,Hq,Sq,D]."""
+    _check(q, "q")
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, S, D]")
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    _check(k, "k", (B, Hkv, Sk, D))
+    _check(v, "v", (B, Hkv, Sk, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    st = lib().rope_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv,
+                             Sq, Sk, D, float(rope_base), int(pos_offset), int(bool(causal)),
+                             _stream(stream))
+    _raise(st, "rope_attn_fwd")
+    return out
+
+
+def rope_attn_rotate(x, rope_base: float, pos_offset: int = 0, out=None, stream=None):
+    """RoPE-rotate x [B,H,S,D] at positions pos_offset + s; out may be x (in place)."""
+    _check(x, "x")
+    B, H, S, D = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(out, "out", x.shape)
+    st = lib().rope_attn_rotate(x.data_ptr(), out.data_ptr(), B, H, S, D, float(rope_base),
+                                int(pos_offset), _stream(stream))
+    _raise(st, "rope_attn_rotate")
+    return out
+
+
+def rope_attn_decode(q, k_cache_rot, v_cache, rope_base: float, pos: int, n_splits: int = 0,
+                     out=None, stream=None):
+    """One decode step. q [B,Hq,1,D]; caches [B,Hkv,Sk,D] (keys pre-rotated); returns out."""
+    _check(q, "q")
+    B, Hq, one, D = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query row per head")
+    Hkv, Sk = k_cache_rot.shape[1], k_cache_rot.shape[2]
+    _check(k_cache_rot, "k_cache_rot", (B, Hkv, Sk, D))
+    _check(v_cache, "v_cache", (B, Hkv, Sk, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    st = lib().rope_attn_decode(q.data_ptr(), k_cache_rot.data_ptr(), v_cache.data_ptr(),
+                                out.data_ptr(), B, Hq, Hkv, Sk, D, float(rope_base), int(pos),
+                                int(n_splits), _stream(stream))
+    _raise(st, "rope_attn_decode")
+    return out
+
+
+def rope_attn_decode_auto_splits(B, Hq, Hkv, Sk, D, pos) -> int:
+    return lib().rope_attn_decode_auto_splits(B, Hq, Hkv, Sk, D, pos)
+
+
+def rope_attn_get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the sticky kernel status."""
+    return lib().rope_attn_get_device_status(_stream(stream))
+
+
+def rope_attn_set_wait_limit(limit: int) -> int:
+    return lib().rope_attn_set_wait_limit(int(limit))
+
+
+def rope_attn_version() -> int:
+    return lib().rope_attn_version()

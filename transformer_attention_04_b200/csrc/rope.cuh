@@ -1,0 +1,92 @@
+// RoPE on sm_100a: the rotation angles and the HBM-bound rotation of whole K (or any
+// [rows, S, D] bf16 tensor).
+//
+// Rotary Position Embeddings as in "Transformer Architecture & Self-Attention
+// Mechanics" (devthesis.com), §3 "Rotary Position Embeddings (RoPE)": the pair
+// (x_2i, x_2i+1) of a row at absolute position m is multiplied by
+// [[cos m*theta_i, -sin m*theta_i], [sin m*theta_i, cos m*theta_i]] with
+// theta_i = base^(-2i/D); the base is a parameter ("Transformer internals: attention
+// without the mysticism", section "Rotary positional embeddings (RoPE)").
+//
+// Angles reach 32767 rad at S = 32768, where a float product alone is off by ~2e-3
+// rad, so theta_i and m*theta_i are formed in fp64 and cos/sin taken in fp64 before
+// narrowing to fp32.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace ra {
+
+__device__ __forceinline__ void rope_cos_sin(long long pos, int i, int D, double log2_base,
+                                             float& c, float& s) {
+  const double theta = exp2(-(2.0 * i / D) * log2_base);  // base^(-2i/D)
+  double sd, cd;
+  sincos(static_cast<double>(pos) * theta, &sd, &cd);
+  c = static_cast<float>(cd);
+  s = static_cast<float>(sd);
+}
+
+// Table of (cos, sin) for `rows` consecutive absolute positions starting at pos0:
+// tab[r * D/2 + i] = (cos, sin)((pos0 + r) * theta_i).
+__global__ void rope_table_kernel(float2* __restrict__ tab, long long pos0, int rows, int D,
+                                  float base) {
+  const double log2_base = log2(static_cast<double>(base));
+  const long long n = static_cast<long long>(rows) * (D / 2);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int r = static_cast<int>(e / (D / 2));
+    const int i = static_cast<int>(e % (D / 2));
+    float c, s;
+    rope_cos_sin(pos0 + r, i, D, log2_base, c, s);
+    tab[e] = make_float2(c, s);
+  }
+}
+
+// Rotate 8 bf16 (4 pairs) given their 4 (cos, sin) pairs; fp32 math, bf16 RNE store.
+__device__ __forceinline__ uint4 rotate8(uint4 x, const float2 (&cs)[4]) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const float x0 = bf16_lo(w[t]), x1 = bf16_hi(w[t]);
+    o[t] = pack_bf16(x0 * cs[t].x - x1 * cs[t].y, x0 * cs[t].y + x1 * cs[t].x);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// x, y: [nrows_total = BH * S, D] bf16, row r at sequence index r % S.
+// kTable: angles from `tab` (row tab_off + s); else computed here at pos0 + s.
+template <bool kTable>
+__global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* __restrict__ x,
+                                                          uint4* __restrict__ y,
+                                                          const float2* __restrict__ tab,
+                                                          long long nrows_total, int S, int D,
+                                                          long long pos0, int tab_off,
+                                                          float base) {
+  const int cpr = D / 8;  // 16-byte chunks per row
+  const long long n = nrows_total * cpr;
+  const double log2_base = kTable ? 0.0 : log2(static_cast<double>(base));
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long row = e / cpr;
+    const int chunk = static_cast<int>(e - row * cpr);
+    const int s = static_cast<int>(row % S);
+    const uint4 v = __ldg(x + e);
+    float2 cs[4];
+    if (kTable) {
+      const float4* t4 =
+          reinterpret_cast<const float4*>(tab + static_cast<long long>(tab_off + s) * (D / 2) + chunk * 4);
+      const float4 a = __ldg(t4), b = __ldg(t4 + 1);
+      cs[0] = make_float2(a.x, a.y);
+      cs[1] = make_float2(a.z, a.w);
+      cs[2] = make_float2(b.x, b.y);
+      cs[3] = make_float2(b.z, b.w);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) rope_cos_sin(pos0 + s, chunk * 4 + t, D, log2_base, cs[t].x, cs[t].y);
+    }
+    y[e] = rotate8(v, cs);
+  }
+}
+
+}  // namespace ra

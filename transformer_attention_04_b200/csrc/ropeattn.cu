@@ -1,0 +1,381 @@
+// libropeattn host side: the C-ABI entry points declared in include/ropeattn.h.
+// Validation, workspace, TMA descriptors and launches; every step of the attention
+// itself runs in the kernels of rope.cuh, attn_fwd_sm100.cuh and decode.cuh.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/ropeattn.h"
+#include "attn_fwd_sm100.cuh"
+#include "decode.cuh"
+#include "rope.cuh"
+
+namespace {
+
+__device__ unsigned int g_device_status;  // sticky kernel status (ra::kStatus*)
+
+std::atomic<long long> g_wait_limit{1LL << 26};
+thread_local char g_last_cuda_error[256] = "";
+
+struct DeviceState {
+  bool ready = false;
+  unsigned int* status = nullptr;
+  int num_sms = 0;
+  bool sm100 = false;
+};
+constexpr int kMaxDevices = 64;
+DeviceState g_devices[kMaxDevices];
+std::mutex g_devices_mu;
+
+ra_status cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what,
+                cudaGetErrorString(e));
+  return RA_ERR_CUDA;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// Per-device set-up, once per device with that device current: the address of the status
+// word, the SM count, the architecture check and the kernels' shared-memory limits.
+ra_status device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return RA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_devices_mu);
+  DeviceState& st = g_devices[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    st.sm100 = (major == 10 && minor == 0);
+    st.num_sms = sms;
+    if (st.sm100) {
+      void* p = nullptr;
+      if ((e = cudaGetSymbolAddress(&p, g_device_status)) != cudaSuccess)
+        return cuda_fail(e, "cudaGetSymbolAddress(status)");
+      st.status = static_cast<unsigned int*>(p);
+      if ((e = set_smem(ra::attn_fwd_sm100_kernel<64>, ra::FwdCfg<64>::SMEM)) != cudaSuccess ||
+          (e = set_smem(ra::attn_fwd_sm100_kernel<128>, ra::FwdCfg<128>::SMEM)) != cudaSuccess ||
+          (e = set_smem(ra::decode_split_kernel<64>, ra::DecCfg<64>::SMEM)) != cudaSuccess ||
+          (e = set_smem(ra::decode_split_kernel<128>, ra::DecCfg<128>::SMEM)) != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    st.ready = true;
+  }
+  if (!st.sm100) return RA_ERR_UNSUPPORTED;
+  *out = &st;
+  return RA_OK;
+}
+
+// cuTensorMapEncodeTiled from the driver, found once through the runtime (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a contiguous [BH, S, D] bf16 tensor: dims (D, S, BH), box (64, box_rows, 1),
+// 128-byte swizzle; rows past S read as zero.
+ra_status make_map(CUtensorMap* m, const void* ptr, int D, int S, long long BH, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "cuTensorMapEncodeTiled entry point not found");
+    return RA_ERR_CUDA;
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(S) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return RA_ERR_CUDA;
+  }
+  return RA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int grid_for(long long work_items, int threads, int num_sms) {
+  const long long blocks = (work_items + threads - 1) / threads;
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(blocks, num_sms * 16LL)));
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+int decode_splits(int B, int Hkv, int G, int L, int num_sms, int requested) {
+  const int max_splits = std::max(1, (L + 63) / 64);
+  if (requested > 0) return std::min(requested, max_splits);
+  const long long base = static_cast<long long>(B) * Hkv * ((G + 7) / 8);
+  const double slots = 2.0 * num_sms;  // two decode CTAs fit on one SM
+  int best = 1;
+  double best_eff = -1.0;
+  for (int s = 1; s <= std::min(max_splits, 32); ++s) {
+    const double waves = base * s / slots;
+    if (waves < 1.0 && s < max_splits && s < 32) continue;
+    const double eff = waves / std::ceil(waves);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = s;
+    }
+    if (waves >= 2.0 && eff >= 0.95) break;
+  }
+  return best;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rope_attn_version(void) { return 100; }
+
+long long rope_attn_set_wait_limit(long long limit) {
+  if (limit < 0) return g_wait_limit.load();
+  return g_wait_limit.exchange(limit);
+}
+
+const char* rope_attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* rope_attn_status_string(int status) {
+  switch (status) {
+    case RA_OK: return "ok";
+    case RA_ERR_INVALID_ARG: return "invalid argument";
+    case RA_ERR_UNSUPPORTED: return "unsupported";
+    case RA_ERR_CUDA: return g_last_cuda_error[0] ? g_last_cuda_error : "CUDA error";
+    case RA_ERR_DEVICE_TIMEOUT: return "a kernel wait ran out (device timeout)";
+    default: return "unknown status";
+  }
+}
+
+ra_status rope_attn_get_device_status(ra_stream_t stream) {
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int v = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  if ((e = cudaMemcpy(&v, ds->status, sizeof(v), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "read status");
+  const unsigned int zero = 0;
+  if ((e = cudaMemcpy(ds->status, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
+    return cuda_fail(e, "clear status");
+  return (v & ra::kStatusTimeout) ? RA_ERR_DEVICE_TIMEOUT : RA_OK;
+}
+
+ra_status rope_attn_rotate(const void* x, void* x_rot, int B, int H, int S, int D,
+                           float rope_base, int pos_offset, ra_stream_t stream) {
+  if (!x || !x_rot || !aligned16(x) || !aligned16(x_rot)) return RA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || S < 1 || D < 8 || D > 256 || D % 8) return RA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base) || pos_offset < 0) return RA_ERR_INVALID_ARG;
+  if (static_cast<long long>(pos_offset) + S > 0x7fffffffLL) return RA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * H * S;
+  const size_t bytes = static_cast<size_t>(rows) * D * 2;
+  if (x != x_rot && overlap(x, bytes, x_rot, bytes)) return RA_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ra::rope_rotate_kernel<false><<<grid_for(rows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(x_rot), nullptr, rows, S, D, pos_offset,
+      0, rope_base);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "rope_rotate launch");
+}
+
+ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                        int Hkv, int Sq, int Sk, int D, float rope_base, int pos_offset,
+                        int causal, ra_stream_t stream) {
+  if (!q || !k || !v || !out) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return RA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || D < 1) return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
+  if (causal && Sq > Sk) return RA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base) || pos_offset < 0) return RA_ERR_INVALID_ARG;
+  if (static_cast<long long>(pos_offset) + std::max(Sq, Sk) > 0x7fffffffLL) return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const size_t qbytes = static_cast<size_t>(B) * Hq * Sq * D * 2;
+  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
+  if (overlap(out, qbytes, q, qbytes) || overlap(out, qbytes, k, kbytes) ||
+      overlap(out, qbytes, v, kbytes))
+    return RA_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  const int n_slots = (G % 2 == 0) ? 2 : 1;
+  const int n_qtiles = (Sq + 127) / 128;
+  const long long n_units = static_cast<long long>(n_qtiles) * B * Hkv * (G / n_slots);
+  if (n_units > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL)
+    return RA_ERR_UNSUPPORTED;
+
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  // workspace: rotated keys, then the (cos, sin) table for positions
+  // pos_offset + tab_lo .. pos_offset + Sk - 1 (covers every query and key position)
+  const int tab_lo = std::min(0, Sk - Sq);
+  const int tab_len = Sk - tab_lo;
+  const size_t krot_bytes = (kbytes + 255) & ~static_cast<size_t>(255);
+  const size_t tab_bytes = static_cast<size_t>(tab_len) * (D / 2) * sizeof(float2);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, krot_bytes + tab_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+  void* k_rot = ws;
+  float2* tab = reinterpret_cast<float2*>(static_cast<char*>(ws) + krot_bytes);
+
+  // a1: angles -> (cos, sin) table;  a2: K -> K' once
+  ra::rope_table_kernel<<<grid_for(static_cast<long long>(tab_len) * (D / 2), 256, ds->num_sms),
+                          256, 0, s>>>(tab, static_cast<long long>(pos_offset) + tab_lo, tab_len,
+                                       D, rope_base);
+  const long long krows = static_cast<long long>(B) * Hkv * Sk;
+  ra::rope_rotate_kernel<true><<<grid_for(krows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
+      static_cast<const uint4*>(k), static_cast<uint4*>(k_rot), tab, krows, Sk, D, 0, -tab_lo,
+      rope_base);
+
+  CUtensorMap tq, tk, tv;
+  rs = make_map(&tq, q, D, Sq, static_cast<long long>(B) * Hq, 128);
+  if (rs == RA_OK) rs = make_map(&tk, k_rot, D, Sk, static_cast<long long>(B) * Hkv, 128);
+  if (rs == RA_OK) rs = make_map(&tv, v, D, Sk, static_cast<long long>(B) * Hkv, 128);
+  if (rs == RA_OK) {
+    ra::FwdParams p;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.tab = tab;
+    p.status = ds->status;
+    p.wait_limit = g_wait_limit.load();
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Sk = Sk;
+    p.G = G;
+    p.n_slots = n_slots;
+    p.ppg = G / n_slots;
+    p.n_qtiles = n_qtiles;
+    p.causal = causal ? 1 : 0;
+    p.q_tab_off = (Sk - Sq) - tab_lo;
+    p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+    const dim3 grid(static_cast<unsigned>(n_units));
+    if (D == 64)
+      ra::attn_fwd_sm100_kernel<64><<<grid, 384, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
+    else
+      ra::attn_fwd_sm100_kernel<128><<<grid, 384, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) rs = cuda_fail(e, "attn_fwd launch");
+  }
+  cudaError_t ef = cudaFreeAsync(ws, s);
+  if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
+  return rs;
+}
+
+int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos) {
+  (void)D;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sk < 1 || pos < 0 || Hq % Hkv) return 0;
+  DeviceState* ds = nullptr;
+  const int sms = (device_state(&ds) == RA_OK) ? ds->num_sms : 148;
+  const int L = std::min(Sk, pos + 1);
+  return decode_splits(B, Hkv, Hq / Hkv, L, sms, 0);
+}
+
+ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const void* v_cache,
+                           void* out, int B, int Hq, int Hkv, int Sk, int D, float rope_base,
+                           int pos, int n_splits, ra_stream_t stream) {
+  if (!q || !k_cache_rot || !v_cache || !out) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache_rot) || !aligned16(v_cache) || !aligned16(out))
+    return RA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sk < 1 || D < 1 || pos < 0 || n_splits < 0)
+    return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const size_t qbytes = static_cast<size_t>(B) * Hq * D * 2;
+  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
+  if (overlap(out, qbytes, q, qbytes) || overlap(out, qbytes, k_cache_rot, kbytes) ||
+      overlap(out, qbytes, v_cache, kbytes))
+    return RA_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  const int hblocks = (G + 7) / 8;
+  if (static_cast<long long>(B) * Hkv * hblocks > 65535) return RA_ERR_UNSUPPORTED;
+
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  const int L = std::min(Sk, pos + 1);
+  int splits = decode_splits(B, Hkv, G, L, ds->num_sms, n_splits);
+  const int chunk = ((L + splits - 1) / splits + 63) / 64 * 64;
+  splits = (L + chunk - 1) / chunk;
+
+  const size_t po_bytes = static_cast<size_t>(B) * Hq * splits * D * sizeof(float);
+  const size_t pml_bytes = static_cast<size_t>(B) * Hq * splits * sizeof(float2);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, po_bytes + pml_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(decode partials)");
+
+  CUtensorMap tk, tv;
+  rs = make_map(&tk, k_cache_rot, D, Sk, static_cast<long long>(B) * Hkv, 64);
+  if (rs == RA_OK) rs = make_map(&tv, v_cache, D, Sk, static_cast<long long>(B) * Hkv, 64);
+  if (rs == RA_OK) {
+    ra::DecParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.part_o = static_cast<float*>(ws);
+    p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + po_bytes);
+    p.status = ds->status;
+    p.wait_limit = g_wait_limit.load();
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.Sk = Sk;
+    p.L = L;
+    p.pos = pos;
+    p.n_splits = splits;
+    p.chunk = chunk;
+    p.hblocks = hblocks;
+    p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+    p.rope_base = rope_base;
+    const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(B * Hkv * hblocks));
+    if (D == 64)
+      ra::decode_split_kernel<64><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
+    else
+      ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
+    ra::decode_combine_kernel<<<static_cast<unsigned>(B * Hq), D, 0, s>>>(
+        p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(out), splits, D);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) rs = cuda_fail(e, "decode launch");
+  }
+  cudaError_t ef = cudaFreeAsync(ws, s);
+  if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(decode partials)");
+  return rs;
+}
+
+}  // extern "C"
