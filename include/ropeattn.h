@@ -119,6 +119,17 @@ RA_API ra_status rope_attn_get_device_status(ra_stream_t stream);
  */
 RA_API long long rope_attn_set_wait_limit(long long limit);
 
+/*
+ * Kernel timing for profiling. While enabled, every rope_attn_fwd call records a pair of
+ * CUDA events on its stream around its attention kernel, and every rope_attn_decode call
+ * around its split kernel. rope_attn_profile_read(which = 0: prefill attention kernel,
+ * 1: decode split kernel) waits for the recorded events, returns the summed kernel time in
+ * milliseconds and the number of launches, and starts a new count. Enabling (or disabling)
+ * also starts a new count. Meant for one device at a time; not for concurrent callers.
+ */
+RA_API ra_status rope_attn_profile_enable(int enable);
+RA_API ra_status rope_attn_profile_read(int which, double* total_ms, int* launches);
+
 /* Text of a status code; the last CUDA error string for RA_ERR_CUDA. */
 RA_API const char* rope_attn_status_string(int status);
 RA_API const char* rope_attn_last_cuda_error(void);

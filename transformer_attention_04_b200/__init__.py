@@ -16,6 +16,8 @@ from ._lib import (  # noqa: F401
     rope_attn_decode_auto_splits,
     rope_attn_fwd,
     rope_attn_get_device_status,
+    rope_attn_profile_enable,
+    rope_attn_profile_read,
     rope_attn_rotate,
     rope_attn_set_wait_limit,
     rope_attn_version,

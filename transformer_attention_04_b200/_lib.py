@@ -29,6 +29,8 @@ SIGNATURES = {
     "rope_attn_status_string": (ctypes.c_char_p, [_I]),
     "rope_attn_last_cuda_error": (ctypes.c_char_p, []),
     "rope_attn_version": (_I, []),
+    "rope_attn_profile_enable": (_I, [_I]),
+    "rope_attn_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I)]),
 }
 
 _lib = None
@@ -146,3 +148,15 @@ def rope_attn_set_wait_limit(limit: int) -> int:
 
 def rope_attn_version() -> int:
     return lib().rope_attn_version()
+
+
+def rope_attn_profile_enable(enable: bool = True) -> None:
+    _raise(lib().rope_attn_profile_enable(int(bool(enable))), "rope_attn_profile_enable")
+
+
+def rope_attn_profile_read(which: int):
+    """(summed kernel ms, launches) since the last read; which 0 = prefill, 1 = decode."""
+    ms, n = ctypes.c_double(0.0), ctypes.c_int(0)
+    _raise(lib().rope_attn_profile_read(int(which), ctypes.byref(ms), ctypes.byref(n)),
+           "rope_attn_profile_read")
+    return ms.value, n.value

@@ -12,6 +12,8 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/ropeattn.h"
 #include "attn_fwd_sm100.cuh"
@@ -23,6 +25,44 @@ namespace {
 __device__ unsigned int g_device_status;  // sticky kernel status (ra::kStatus*)
 
 std::atomic<long long> g_wait_limit{1LL << 26};
+
+// Kernel-time profiling: event pairs recorded around the main kernel of each call.
+struct ProfKind {
+  int device = -1;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev;
+  size_t used = 0;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+ProfKind g_prof[2];  // 0: prefill attention kernel, 1: decode split kernel
+
+// Records the start event (returns the pair index) or -1 when profiling is off.
+int prof_start(int kind, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (!g_prof_on) return -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  ProfKind& pk = g_prof[kind];
+  if (pk.device != dev) {
+    if (pk.used) return -1;  // one device per profiling session
+    for (auto& e : pk.ev) { cudaEventDestroy(e.first); cudaEventDestroy(e.second); }
+    pk.ev.clear();
+    pk.device = dev;
+  }
+  if (pk.used == pk.ev.size()) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess) return -1;
+    if (cudaEventCreate(&b) != cudaSuccess) { cudaEventDestroy(a); return -1; }
+    pk.ev.emplace_back(a, b);
+  }
+  if (cudaEventRecord(pk.ev[pk.used].first, s) != cudaSuccess) return -1;
+  return static_cast<int>(pk.used++);
+}
+void prof_stop(int kind, int idx, cudaStream_t s) {
+  if (idx < 0) return;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  cudaEventRecord(g_prof[kind].ev[idx].second, s);
+}
 thread_local char g_last_cuda_error[256] = "";
 
 struct DeviceState {
@@ -166,6 +206,31 @@ extern "C" {
 
 int rope_attn_version(void) { return 100; }
 
+ra_status rope_attn_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  g_prof_on = enable != 0;
+  g_prof[0].used = g_prof[1].used = 0;
+  return RA_OK;
+}
+
+ra_status rope_attn_profile_read(int which, double* total_ms, int* launches) {
+  if ((which != 0 && which != 1) || !total_ms || !launches) return RA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  ProfKind& pk = g_prof[which];
+  double sum = 0.0;
+  for (size_t i = 0; i < pk.used; ++i) {
+    cudaError_t e = cudaEventSynchronize(pk.ev[i].second);
+    float ms = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pk.ev[i].first, pk.ev[i].second);
+    if (e != cudaSuccess) return cuda_fail(e, "profile events");
+    sum += ms;
+  }
+  *total_ms = sum;
+  *launches = static_cast<int>(pk.used);
+  pk.used = 0;
+  return RA_OK;
+}
+
 long long rope_attn_set_wait_limit(long long limit) {
   if (limit < 0) return g_wait_limit.load();
   return g_wait_limit.exchange(limit);
@@ -288,10 +353,12 @@ ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     p.q_tab_off = (Sk - Sq) - tab_lo;
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
     const dim3 grid(static_cast<unsigned>(n_units));
+    const int pi = prof_start(0, s);
     if (D == 64)
       ra::attn_fwd_sm100_kernel<64><<<grid, 384, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
     else
       ra::attn_fwd_sm100_kernel<128><<<grid, 384, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
+    prof_stop(0, pi, s);
     e = cudaGetLastError();
     if (e != cudaSuccess) rs = cuda_fail(e, "attn_fwd launch");
   }
@@ -364,10 +431,12 @@ ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const void* v
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
     p.rope_base = rope_base;
     const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(B * Hkv * hblocks));
+    const int pi = prof_start(1, s);
     if (D == 64)
       ra::decode_split_kernel<64><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
     else
       ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
+    prof_stop(1, pi, s);
     ra::decode_combine_kernel<<<static_cast<unsigned>(B * Hq), D, 0, s>>>(
         p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(out), splits, D);
     e = cudaGetLastError();
