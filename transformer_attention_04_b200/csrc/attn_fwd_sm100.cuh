@@ -38,6 +38,19 @@
 
 namespace ra {
 
+#ifdef RA_TRACE
+// Per-phase clock64() stamps of CTAs 0-1 for the first 64 KV tiles (profiling builds only).
+__device__ unsigned long long g_trace[2][16][64];
+#define RA_STAMP(ev, j)                                                         \
+  do {                                                                          \
+    if (blockIdx.x < 2 && (j) < 64) g_trace[blockIdx.x][(ev)][(j)] = clock64(); \
+  } while (0)
+#else
+#define RA_STAMP(ev, j) \
+  do {                  \
+  } while (0)
+#endif
+
 struct FwdParams {
   __nv_bfloat16* out;   // [B, Hq, Sq, D]
   const float2* tab;    // RoPE (cos, sin) table, D/2 entries per position
@@ -58,11 +71,12 @@ struct FwdCfg {
   static constexpr int KB = D / 64;                  // 128-byte column blocks per row
   static constexpr int BLK = 128 * 128;              // bytes of one 128-row column block
   static constexpr int TILE = 128 * D * 2;           // bytes of one 128 x D bf16 tile
-  static constexpr int NST = (D == 128) ? 2 : 4;     // K/V ring depth
+  // K and V tiles stream through one ring in the order K0 V0 K1 V1 ...: 5 slots at D = 128
+  // (2.5 KV tiles of look-ahead; 2 Q tiles + 5 slots = 224 KB of shared memory).
+  static constexpr int NSLOT = (D == 128) ? 5 : 8;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * TILE;
-  static constexpr int OFF_V = OFF_K + NST * TILE;
-  static constexpr int OFF_BAR = OFF_V + NST * TILE;
+  static constexpr int OFF_RING = OFF_Q + 2 * TILE;
+  static constexpr int OFF_BAR = OFF_RING + NSLOT * TILE;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;  // barriers + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns: S/P of slot s at 128*s, O of slot s at 256 + D*s
@@ -70,14 +84,58 @@ struct FwdCfg {
   __device__ static constexpr uint32_t col_o(int s) { return 256u + static_cast<uint32_t>(D * s); }
   // barrier indices (8 bytes each)
   static constexpr int B_QFULL = 0, B_QREADY = 2, B_SFULL = 4, B_PFULL = 6, B_OFULL = 8,
-                       B_DRAIN = 10, B_KFULL = 11, B_KEMPTY = 11 + NST, B_VFULL = 11 + 2 * NST,
-                       B_VEMPTY = 11 + 3 * NST, N_BAR = 11 + 4 * NST;
+                       B_DRAIN = 10, B_FULL = 11, B_EMPTY = 11 + NSLOT, N_BAR = 11 + 2 * NSLOT;
   static constexpr int OFF_TMEM_SLOT = 8 * N_BAR;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
   static_assert(OFF_ABORT + 4 <= 512, "barrier area");
+  static_assert(SMEM <= 232448, "shared memory per block");
 };
 
-template <int D>
+// P = 2^(s * sl2 - m) for one 128-column row of S held in registers; writes the bf16 P
+// over the first 64 TMEM columns at tS and returns the row sum of the fp32 values.
+// Pairs go through one packed FMA; kEmu of every 4 pairs use the FMA-pipe exponential.
+template <int kEmu>
+__device__ __forceinline__ float softmax_p_store(const uint32_t* sr, float sl2, float m,
+                                                 uint32_t tS) {
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m, -m);
+  uint64_t acc2[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c2 = 0; c2 < 32; ++c2) {
+      const int c = h * 64 + 2 * c2;
+      const uint64_t x2 =
+          f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
+      uint64_t p2;
+      if ((c2 & 3) < kEmu) {
+        p2 = exp2_poly_x2(x2);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p2 = f2_pack(ex2(x0), ex2(x1));
+      }
+      acc2[c2 & 3] = f2_add(acc2[c2 & 3], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[c2] = pack_bf16(p0, p1);
+    }
+    tmem_st32(tS + 32 * h, pk);
+  }
+  const uint64_t a = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+  float a0, a1;
+  f2_unpack(a, a0, a1);
+  return a0 + a1;
+}
+
+#ifndef RA_EMU_PAIRS
+#define RA_EMU_PAIRS 1
+#endif
+
+// kEmuPairs: of every 4 column pairs of an unmasked tile, how many take the FMA-pipe
+// exponential (0 = all on the MUFU).
+template <int D, int kEmuPairs = RA_EMU_PAIRS>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -87,7 +145,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V;
+  const uint32_t sQ = base + C::OFF_Q, sRing = base + C::OFF_RING;
   const uint32_t sBar = base + C::OFF_BAR;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + C::OFF_ABORT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + C::OFF_TMEM_SLOT);
@@ -114,17 +172,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(C::B_QFULL + s), 1);
-      mbar_init(bar(C::B_QREADY + s), 128);
+      mbar_init(bar(C::B_QREADY + s), 4);  // one arrival per softmax warp
       mbar_init(bar(C::B_SFULL + s), 1);
-      mbar_init(bar(C::B_PFULL + s), 128);
+      mbar_init(bar(C::B_PFULL + s), 4);
       mbar_init(bar(C::B_OFULL + s), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
-    for (int i = 0; i < C::NST; ++i) {
-      mbar_init(bar(C::B_KFULL + i), 1);
-      mbar_init(bar(C::B_KEMPTY + i), 1);
-      mbar_init(bar(C::B_VFULL + i), 1);
-      mbar_init(bar(C::B_VEMPTY + i), 1);
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(bar(C::B_FULL + i), 1);
+      mbar_init(bar(C::B_EMPTY + i), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -144,50 +200,40 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = *tmem_slot;
 
   // Register split: launched at 168 per thread (384 x 168 = 64512); the control
-  // warpgroup gives back to 56, the two softmax warpgroups take 224
-  // (128 x 56 + 256 x 224 = 64512).
+  // warpgroup gives back to 80, the two softmax warpgroups take 208
+  // (128 x 80 + 256 x 208 = 63488 <= 64512).
   if (warp < 4) {
-  regs_dec<56>();
+  regs_dec<80>();
   if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
-      int issued = 0;
       for (int s = 0; s < ns; ++s) {
         mbar_expect_tx(bar(C::B_QFULL + s), C::TILE);
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_3d(sQ + s * C::TILE + kb * C::BLK, &tm_q, kb * 64, q0, b * p.Hq + h0 + s,
                       bar(C::B_QFULL + s));
       }
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % C::NST;
-        const uint32_t ph = (j / C::NST) & 1;
-        if (j >= C::NST &&
-            !mbar_wait(bar(C::B_KEMPTY + st), ph ^ 1, p.wait_limit, abort_flag, p.status))
+      // ring item i: tile i/2 of K (i even) or V (i odd), in slot i % NSLOT
+      int issued = 0;
+      for (int i = 0; i < 2 * n_kv; ++i) {
+        const int sl = i % C::NSLOT;
+        if (!(i & 1)) RA_STAMP(14, i >> 1);
+        if (i >= C::NSLOT && !mbar_wait(bar(C::B_EMPTY + sl), ((i / C::NSLOT) - 1) & 1,
+                                        p.wait_limit, abort_flag, p.status))
           break;
-        mbar_expect_tx(bar(C::B_KFULL + st), C::TILE);
+        RA_STAMP(12 + (i & 1), i >> 1);
+        mbar_expect_tx(bar(C::B_FULL + sl), C::TILE);
+        const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sK + st * C::TILE + kb * C::BLK, &tm_k, kb * 64, j * 128, kv_bh,
-                      bar(C::B_KFULL + st));
-        if (j >= C::NST &&
-            !mbar_wait(bar(C::B_VEMPTY + st), ph ^ 1, p.wait_limit, abort_flag, p.status)) {
-          issued = -(j + 1);  // K of tile j in flight, V not
-          break;
-        }
-        mbar_expect_tx(bar(C::B_VFULL + st), C::TILE);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sV + st * C::TILE + kb * C::BLK, &tm_v, kb * 64, j * 128, kv_bh,
-                      bar(C::B_VFULL + st));
-        issued = j + 1;
+          tma_load_3d(sRing + sl * C::TILE + kb * C::BLK, map, kb * 64, (i >> 1) * 128, kv_bh,
+                      bar(C::B_FULL + sl));
+        issued = i + 1;
       }
       if (*abort_flag) {
         // let every copy this thread started land before the CTA can exit
         for (int s = 0; s < ns; ++s) mbar_drain(bar(C::B_QFULL + s), 0);
-        const int nk = issued >= 0 ? issued : -issued;
-        const int nv = issued >= 0 ? issued : -issued - 1;
-        for (int j = max(0, nk - C::NST); j < nk; ++j)
-          mbar_drain(bar(C::B_KFULL + j % C::NST), (j / C::NST) & 1);
-        for (int j = max(0, nv - C::NST); j < nv; ++j)
-          mbar_drain(bar(C::B_VFULL + j % C::NST), (j / C::NST) & 1);
+        for (int i = max(0, issued - C::NSLOT); i < issued; ++i)
+          mbar_drain(bar(C::B_FULL + i % C::NSLOT), (i / C::NSLOT) & 1);
       }
     }
   } else if (warp == 1) {
@@ -195,75 +241,87 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc_bf16(128, 128, 0, 0);  // Q, K both K-major
       constexpr uint32_t kIdescO = umma_idesc_bf16(128, D, 0, 1);    // V is MN-major
-      auto issue_s = [&](int s, int st) {
+      // descriptors of the Q tiles and of ring slot 0; other slots / k-steps add offsets >> 4
+      const uint64_t dq0 = umma_smem_desc(sQ, 16, 1024, kLayoutSW128);
+      const uint64_t dk0 = umma_smem_desc(sRing, 16, 1024, kLayoutSW128);
+      const uint64_t dv0 = umma_smem_desc(sRing, C::BLK, 1024, kLayoutSW128);
+      auto issue_s = [&](int s, int sl) {
         const uint32_t d_t = tmem + C::col_s(s);
+        const uint64_t a = dq0 + static_cast<uint64_t>((s * C::TILE) >> 4);
+        const uint64_t bq = dk0 + static_cast<uint64_t>((sl * C::TILE) >> 4);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t o = (k >> 2) * C::BLK + (k & 3) * 32;
-          const uint64_t ad = umma_smem_desc(sQ + s * C::TILE + o, 16, 1024, kLayoutSW128);
-          const uint64_t bd = umma_smem_desc(sK + st * C::TILE + o, 16, 1024, kLayoutSW128);
-          umma_ss(d_t, ad, bd, kIdescS, k > 0 ? 1u : 0u);
+          const uint64_t o = static_cast<uint64_t>(((k >> 2) * C::BLK + (k & 3) * 32) >> 4);
+          umma_ss(d_t, a + o, bq + o, kIdescS, k > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int s, int st, bool acc) {
+      auto issue_pv = [&](int s, int sl, bool acc) {
         const uint32_t d_t = tmem + C::col_o(s);
         const uint32_t a_t = tmem + C::col_s(s);
+        const uint64_t bv = dv0 + static_cast<uint64_t>((sl * C::TILE) >> 4);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {  // 128 keys, 16 per MMA
-          const uint64_t bd =
-              umma_smem_desc(sV + st * C::TILE + k * 2048, C::BLK, 1024, kLayoutSW128);
-          umma_ts(d_t, a_t + 8 * k, bd, kIdescO, (acc || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < 8; ++k)  // 128 keys, 16 per MMA
+          umma_ts(d_t, a_t + 8 * k, bv + static_cast<uint64_t>((k * 2048) >> 4), kIdescO,
+                  (acc || k > 0) ? 1u : 0u);
       };
+      auto kslot = [](int j) { return (2 * j) % C::NSLOT; };
+      auto kpar = [](int j) { return static_cast<uint32_t>(((2 * j) / C::NSLOT) & 1); };
+      auto vslot = [](int j) { return (2 * j + 1) % C::NSLOT; };
+      auto vpar = [](int j) { return static_cast<uint32_t>(((2 * j + 1) / C::NSLOT) & 1); };
       const long long lim = p.wait_limit;
       bool ok = mbar_wait(bar(C::B_QREADY + 0), 0, lim, abort_flag, p.status) &&
-                mbar_wait(bar(C::B_KFULL + 0), 0, lim, abort_flag, p.status);
+                mbar_wait(bar(C::B_FULL + kslot(0)), kpar(0), lim, abort_flag, p.status);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
+        issue_s(0, kslot(0));
         umma_commit(bar(C::B_SFULL + 0));
         if (ns == 2) {
           ok = mbar_wait(bar(C::B_QREADY + 1), 0, lim, abort_flag, p.status);
           if (ok) {
             tc_fence_after();
-            issue_s(1, 0);
+            issue_s(1, kslot(0));
             umma_commit(bar(C::B_SFULL + 1));
           }
         }
-        umma_commit(bar(C::B_KEMPTY + 0));
+        umma_commit(bar(C::B_EMPTY + kslot(0)));
       }
       for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j % C::NST;
-        const uint32_t ph = (j / C::NST) & 1;
         const bool has_next = j + 1 < n_kv;
-        const int st1 = (j + 1) % C::NST;
-        const uint32_t ph1 = ((j + 1) / C::NST) & 1;
+        RA_STAMP(0, j);
         if (!mbar_wait(bar(C::B_PFULL + 0), j & 1, lim, abort_flag, p.status) ||
-            !mbar_wait(bar(C::B_VFULL + st), ph, lim, abort_flag, p.status))
+            !mbar_wait(bar(C::B_FULL + vslot(j)), vpar(j), lim, abort_flag, p.status))
           break;
         tc_fence_after();
-        issue_pv(0, st, j > 0);
+        RA_STAMP(1, j);
+        issue_pv(0, vslot(j), j > 0);
+        RA_STAMP(2, j);
         if (!has_next) umma_commit(bar(C::B_OFULL + 0));
         if (has_next) {
-          if (!mbar_wait(bar(C::B_KFULL + st1), ph1, lim, abort_flag, p.status)) break;
+          if (!mbar_wait(bar(C::B_FULL + kslot(j + 1)), kpar(j + 1), lim, abort_flag, p.status))
+            break;
           tc_fence_after();
-          issue_s(0, st1);
+          RA_STAMP(3, j);
+          issue_s(0, kslot(j + 1));
+          RA_STAMP(4, j);
           umma_commit(bar(C::B_SFULL + 0));
         }
         if (ns == 2) {
           if (!mbar_wait(bar(C::B_PFULL + 1), j & 1, lim, abort_flag, p.status)) break;
           tc_fence_after();
-          issue_pv(1, st, j > 0);
+          RA_STAMP(5, j);
+          issue_pv(1, vslot(j), j > 0);
+          RA_STAMP(6, j);
           if (!has_next) umma_commit(bar(C::B_OFULL + 1));
-          umma_commit(bar(C::B_VEMPTY + st));
+          umma_commit(bar(C::B_EMPTY + vslot(j)));
           if (has_next) {
-            issue_s(1, st1);
+            issue_s(1, kslot(j + 1));
+            RA_STAMP(7, j);
             umma_commit(bar(C::B_SFULL + 1));
-            umma_commit(bar(C::B_KEMPTY + st1));
+            umma_commit(bar(C::B_EMPTY + kslot(j + 1)));
           }
         } else {
-          umma_commit(bar(C::B_VEMPTY + st));
-          if (has_next) umma_commit(bar(C::B_KEMPTY + st1));
+          umma_commit(bar(C::B_EMPTY + vslot(j)));
+          if (has_next) umma_commit(bar(C::B_EMPTY + kslot(j + 1)));
         }
       }
       // every MMA issued above must finish before TMEM is released
@@ -273,7 +331,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   }
   } else {
-  regs_inc<224>();
+  regs_inc<208>();
   if ((warp >> 2) - 1 < ns) {
     // ================================================================ softmax warpgroups
     const int s = (warp >> 2) - 1;
@@ -305,7 +363,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
     fence_proxy_async_smem();
-    mbar_arrive(bar(C::B_QREADY + s));
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(C::B_QREADY + s));
 
     float m = -INFINITY;  // running row max, in log2 units of the scaled score
     float l = 0.f;        // running row sum of 2^(x - m)
@@ -317,6 +376,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         break;
       }
       tc_fence_after();
+      if (lane == 0 && qd == 0) RA_STAMP(8 + 2 * s, j);
       uint32_t sr[128];
       tmem_ld32(tS + 0, sr + 0);
       tmem_ld32(tS + 32, sr + 32);
@@ -334,9 +394,20 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (c > lim_k) sr[c] = 0xff800000u;  // -inf
       }
       // a7: online softmax with a lazily updated reference max
-      float mt = -INFINITY;
+      // tile max of the raw scores: eight independent 3-input max chains, then a tree
+      float mx[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mt = fmaxf(mt, __uint_as_float(sr[c]));
+      for (int k = 0; k < 8; ++k)
+        mx[k] = max3f(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]), __uint_as_float(sr[k + 16]));
+#pragma unroll
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mx[k] = max3f(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[120 + k]));
+      const float mt = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]),
+                             fmaxf(mx[6], mx[7]));
       const float m_new = fmaxf(m, mt * sl2);
       // Keep the old reference unless the max grew by more than 8 (P stays <= 256);
       // O / l is exact for any common reference, so skipping the rescale is lossless.
@@ -356,25 +427,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_st32(tO + cb, o);
         }
       }
-      const float neg_m = -m;
-      float rs = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const int c = h * 64 + 2 * c2;
-          const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, neg_m));
-          rs += p0 + p1;
-          pk[c2] = pack_bf16(p0, p1);
-        }
-        tmem_st32(tS + 32 * h, pk);
-      }
+      // p = 2^(s * log2(e)/sqrt(D) - m) -> bf16 P over the S columns; unmasked tiles send
+      // part of the exponentials to the FMA pipe
+      const float rs = need_mask ? softmax_p_store<0>(sr, sl2, m, tS)
+                                 : softmax_p_store<kEmuPairs>(sr, sl2, m, tS);
       l += rs;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::B_PFULL + s));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_PFULL + s));
+      if (lane == 0 && qd == 0) RA_STAMP(9 + 2 * s, j);
     }
 
     // a10: epilogue O / l -> bf16

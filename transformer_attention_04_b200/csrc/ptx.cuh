@@ -257,6 +257,57 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): element 0 in the low 32 bits.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for two arguments on the FMA pipe (keeps the MUFU free for the other exponentials).
+// x = n + f with n = round(x) taken from the low bits of x + 1.5*2^23 and f in [-1/2, 1/2];
+// 2^f is the cubic fitted by csrc/exp2_poly_fit.py (minimax relative error 7.5e-5), and 2^n
+// is added to the exponent field. Arguments are clamped at -120 (2^-120 is negligible next
+// to a softmax row sum >= 1); callers keep -inf (masked) entries away from this routine.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
+  const uint64_t kMagic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t kNegMagic = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t kNegOne = f2_pack(-1.0f, -1.0f);
+  const uint64_t t = f2_add(xc, kMagic);
+  const uint64_t n = f2_add(t, kNegMagic);
+  const uint64_t f = f2_fma(n, kNegOne, xc);
+  uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
+                      f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
 }  // namespace ra

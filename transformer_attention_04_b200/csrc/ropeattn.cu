@@ -447,4 +447,13 @@ ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const void* v
   return rs;
 }
 
+#ifdef RA_TRACE
+// Profiling builds only: copy the phase stamps of the last prefill launch to the host.
+RA_API int rope_attn_trace_read(void* host, size_t bytes) {
+  if (bytes < sizeof(ra::g_trace)) return RA_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host, ra::g_trace, sizeof(ra::g_trace)) == cudaSuccess ? RA_OK
+                                                                                      : RA_ERR_CUDA;
+}
+#endif
+
 }  // extern "C"
