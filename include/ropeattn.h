@@ -106,8 +106,9 @@ RA_API ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const 
 RA_API int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos);
 
 /*
- * Synchronises `stream`, returns the sticky device status of the current device
- * (RA_OK or RA_ERR_DEVICE_TIMEOUT) and clears it; RA_ERR_CUDA if the sync itself failed.
+ * Synchronises `stream`, returns the sticky device status of the current device and clears
+ * it: RA_OK, RA_ERR_DEVICE_TIMEOUT, or RA_ERR_CUDA if the sync failed or a kernel found its
+ * shared-memory base misaligned (it then did no work; see rope_attn_last_cuda_error).
  */
 RA_API ra_status rope_attn_get_device_status(ra_stream_t stream);
 

@@ -77,7 +77,7 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + 2 * TILE;
   static constexpr int OFF_BAR = OFF_RING + NSLOT * TILE;
-  static constexpr int SMEM = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  static constexpr int SMEM = OFF_BAR + 512;  // the dynamic shared base is 1024-aligned (checked)
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns: S/P of slot s at 128*s, O of slot s at 256 + D*s
   __device__ static constexpr uint32_t col_s(int s) { return 128u * static_cast<uint32_t>(s); }
@@ -130,7 +130,7 @@ __device__ __forceinline__ float softmax_p_store(const uint32_t* sr, float sl2, 
 }
 
 #ifndef RA_EMU_PAIRS
-#define RA_EMU_PAIRS 1
+#define RA_EMU_PAIRS 0
 #endif
 
 // kEmuPairs: of every 4 column pairs of an unmasked tile, how many take the FMA-pipe
@@ -141,10 +141,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = FwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (base - raw);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t base = smem_u32(smem);
+  if (base & 1023u) {  // the 128-byte swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusLayout);
+    return;
+  }
   const uint32_t sQ = base + C::OFF_Q, sRing = base + C::OFF_RING;
   const uint32_t sBar = base + C::OFF_BAR;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + C::OFF_ABORT);
@@ -207,11 +209,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
+      // K/V tiles are re-read by every query tile of their head group: keep them in L2;
+      // each Q tile is read once.
+      const uint64_t pol_keep = l2_policy_evict_last();
+      const uint64_t pol_once = l2_policy_evict_first();
       for (int s = 0; s < ns; ++s) {
         mbar_expect_tx(bar(C::B_QFULL + s), C::TILE);
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sQ + s * C::TILE + kb * C::BLK, &tm_q, kb * 64, q0, b * p.Hq + h0 + s,
-                      bar(C::B_QFULL + s));
+          tma_load_3d_hint(sQ + s * C::TILE + kb * C::BLK, &tm_q, kb * 64, q0, b * p.Hq + h0 + s,
+                           bar(C::B_QFULL + s), pol_once);
       }
       // ring item i: tile i/2 of K (i even) or V (i odd), in slot i % NSLOT
       int issued = 0;
@@ -225,8 +231,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_expect_tx(bar(C::B_FULL + sl), C::TILE);
         const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d(sRing + sl * C::TILE + kb * C::BLK, map, kb * 64, (i >> 1) * 128, kv_bh,
-                      bar(C::B_FULL + sl));
+          tma_load_3d_hint(sRing + sl * C::TILE + kb * C::BLK, map, kb * 64, (i >> 1) * 128, kv_bh,
+                           bar(C::B_FULL + sl), pol_keep);
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -443,6 +449,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (ok && mbar_wait_warp(bar(C::B_OFULL + s), 0, lim, abort_flag, p.status)) {
       tc_fence_after();
       const float inv = 1.0f / l;
+      const uint64_t pol_out = l2_policy_evict_first();
       __nv_bfloat16* orow =
           p.out + (static_cast<long long>(b * p.Hq + h0 + s) * p.Sq + qrow) * D;
 #pragma unroll
@@ -459,7 +466,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             w.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
             w.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
             w.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
-            dst[i] = w;
+            st_global_v4_hint(dst + i, w, pol_out);
           }
         }
       }

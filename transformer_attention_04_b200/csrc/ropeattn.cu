@@ -262,6 +262,11 @@ ra_status rope_attn_get_device_status(ra_stream_t stream) {
   const unsigned int zero = 0;
   if ((e = cudaMemcpy(ds->status, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(e, "clear status");
+  if (v & ra::kStatusLayout) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "kernel shared-memory base was not 1024-byte aligned; no work was done");
+    return RA_ERR_CUDA;
+  }
   return (v & ra::kStatusTimeout) ? RA_ERR_DEVICE_TIMEOUT : RA_OK;
 }
 
@@ -352,6 +357,7 @@ ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     p.causal = causal ? 1 : 0;
     p.q_tab_off = (Sk - Sq) - tab_lo;
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+    // one CTA per work unit; blockIdx order is longest causal extent first
     const dim3 grid(static_cast<unsigned>(n_units));
     const int pi = prof_start(0, s);
     if (D == 64)
