@@ -102,6 +102,33 @@ RA_API ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const 
                            void* out, int B, int Hq, int Hkv, int Sk, int D, float rope_base,
                            int pos, int n_splits, ra_stream_t stream);
 
+/*
+ * rope_attn_decode without any device allocation. No counterpart in the paper: this is a
+ * deployment variant of rope_attn_decode for callers that may not allocate device memory at
+ * call time, for example an inference server that reserves the GPU's memory for its own
+ * pool up front and forbids libraries from taking memory behind its back, or a step that
+ * must not risk an allocation failing (or waiting on the allocator) half-way through.
+ *
+ * Same arguments, layouts and result as rope_attn_decode. The per-split partials go to one
+ * fixed array of 16 MiB (16777216 bytes) that the library keeps in device memory on every
+ * GPU that loads it, until the process exits; the caller still provides q, the caches and
+ * out. Partials take B*Hq*splits*(D*4 + 8) bytes (plus up to 255 of padding): with
+ * n_splits = 0 the split count is lowered until they fit; an explicit n_splits whose
+ * partials do not fit, or sizes that do not fit even with one split, return
+ * RA_ERR_UNSUPPORTED without enqueuing anything (the reason is in
+ * rope_attn_last_cuda_error).
+ *
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture. All calls, on
+ * every stream, share the one array and it keeps the last call's contents: calls whose work
+ * overlaps on the GPU race with each other, so serialise them (one stream, or events).
+ * Nothing in the array needs clearing: every partial is written before it is read.
+ */
+RA_API ra_status rope_attn_decode_noalloc(const void* q, const void* k_cache_rot,
+                                          const void* v_cache, void* out, int B, int Hq, int Hkv,
+                                          int Sk, int D, float rope_base, int pos, int n_splits,
+                                          ra_stream_t stream);
+
 /* Split count rope_attn_decode uses for these sizes when n_splits == 0. */
 RA_API int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos);
 

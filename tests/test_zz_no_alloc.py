@@ -1,0 +1,68 @@
+"""rope_attn_decode_noalloc: the decode step for callers that may not allocate device memory
+while they run it (for instance a serving process that has reserved the GPU's memory for its
+own pool and does not let libraries take more, or a step that must not stall or fail on an
+allocation). The entry keeps its per-split partials in one fixed 16 MiB device array of the
+library instead of memory taken per call.
+
+The test calls the entry through the C ABI twice in a row, on different inputs (so a stale
+partial left by the first call would show in the second), and compares each result with the
+allocating rope_attn_decode within the parity tolerance of the other tests. It also checks
+that a request whose partials cannot fit the array is refused before anything is enqueued.
+The file is named to be collected last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import transformer_attention_04_b200 as ra
+from parity_util import MAX_ABS, REL_RMS, errors
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_BYTES = 16 << 20
+
+
+def _inputs(seed, B, Hq, Hkv, Sk, D):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Hq, 1, D, generator=g).to(torch.bfloat16).cuda()
+    kc = torch.randn(B, Hkv, Sk, D, generator=g).to(torch.bfloat16).cuda()
+    vc = torch.randn(B, Hkv, Sk, D, generator=g).to(torch.bfloat16).cuda()
+    return q, kc, vc
+
+
+def _noalloc(q, kc, vc, base, pos, n_splits):
+    B, Hq, _, D = q.shape
+    Hkv, Sk = kc.shape[1], kc.shape[2]
+    out = torch.empty_like(q)
+    st = ra.lib().rope_attn_decode_noalloc(
+        q.data_ptr(), kc.data_ptr(), vc.data_ptr(), out.data_ptr(), B, Hq, Hkv, Sk, D, base, pos,
+        n_splits, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    return st, out
+
+
+@pytest.mark.parametrize("shape", [(4, 16, 2, 3000, 128, 2999, 0), (2, 8, 8, 777, 64, 700, 3),
+                                   (32, 64, 8, 8192, 128, 8191, 0)])
+def test_noalloc_matches_decode_twice(shape):
+    B, Hq, Hkv, Sk, D, pos, ns = shape
+    base = 500000.0
+    for call, seed in enumerate((11, 12)):
+        q, kc, vc = _inputs(seed, B, Hq, Hkv, Sk, D)
+        ref = ra.rope_attn_decode(q, kc, vc, base, pos, n_splits=ns)
+        st, out = _noalloc(q, kc, vc, base, pos, ns)
+        assert st == ra.RA_OK, ra.lib().rope_attn_last_cuda_error()
+        torch.cuda.synchronize()
+        assert ra.rope_attn_get_device_status() == ra.RA_OK
+        ma, rr = errors(out, ref.double().cpu().numpy())
+        assert ma <= MAX_ABS and rr <= REL_RMS, (call, ma, rr)
+
+
+def test_noalloc_rejects_partials_beyond_scratch():
+    # 64 x 256 heads x 8 splits x (128 x 4 + 8) bytes is about 68 MB, over the 16 MiB array
+    B, Hq, Hkv, Sk, D, splits = 64, 256, 8, 1024, 128, 8
+    q = torch.zeros(B, Hq, 1, D, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(B, Hkv, Sk, D, dtype=torch.bfloat16, device="cuda")
+    st, _ = _noalloc(q, kc, kc.clone(), 500000.0, Sk - 1, splits)
+    assert st == ra.RA_ERR_UNSUPPORTED
+    assert b"scratch" in ra.lib().rope_attn_last_cuda_error()
+    assert B * Hq * splits * (D * 4 + 8) > SCRATCH_BYTES

@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     lib,
     rope_attn_decode,
     rope_attn_decode_auto_splits,
+    rope_attn_decode_noalloc,
     rope_attn_fwd,
     rope_attn_get_device_status,
     rope_attn_profile_enable,

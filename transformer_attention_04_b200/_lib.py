@@ -23,6 +23,7 @@ SIGNATURES = {
     "rope_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "rope_attn_rotate": (_I, [_P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "rope_attn_decode": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "rope_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "rope_attn_decode_auto_splits": (_I, [_I, _I, _I, _I, _I, _I]),
     "rope_attn_get_device_status": (_I, [_P]),
     "rope_attn_set_wait_limit": (_LL, [_LL]),
@@ -130,6 +131,27 @@ def rope_attn_decode(q, k_cache_rot, v_cache, rope_base: float, pos: int, n_spli
                                 out.data_ptr(), B, Hq, Hkv, Sk, D, float(rope_base), int(pos),
                                 int(n_splits), _stream(stream))
     _raise(st, "rope_attn_decode")
+    return out
+
+
+def rope_attn_decode_noalloc(q, k_cache_rot, v_cache, rope_base: float, pos: int,
+                             n_splits: int = 0, out=None, stream=None):
+    """rope_attn_decode with its partials in the library's fixed device scratch (no device
+    allocation per call); see the C header for the size limit and the sharing rules."""
+    _check(q, "q")
+    B, Hq, one, D = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query row per head")
+    Hkv, Sk = k_cache_rot.shape[1], k_cache_rot.shape[2]
+    _check(k_cache_rot, "k_cache_rot", (B, Hkv, Sk, D))
+    _check(v_cache, "v_cache", (B, Hkv, Sk, D))
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    st = lib().rope_attn_decode_noalloc(q.data_ptr(), k_cache_rot.data_ptr(), v_cache.data_ptr(),
+                                        out.data_ptr(), B, Hq, Hkv, Sk, D, float(rope_base),
+                                        int(pos), int(n_splits), _stream(stream))
+    _raise(st, "rope_attn_decode_noalloc")
     return out
 
 

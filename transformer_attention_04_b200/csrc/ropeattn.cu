@@ -200,6 +200,39 @@ int decode_splits(int B, int Hkv, int G, int L, int num_sms, int requested) {
   return best;
 }
 
+// Fixed device scratch of rope_attn_decode_noalloc: the per-split partials live here instead
+// of in memory taken per call. Every device that loads the library holds it until exit.
+constexpr size_t kDecodeScratchBytes = static_cast<size_t>(16) << 20;  // 16 MiB
+__device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+// Device address of the scratch, looked up once per device with that device current (the
+// array's name in host code is only a stand-in for the symbol, not a device address).
+void* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+ra_status decode_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return RA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return RA_OK;
+}
+
+// Bytes of partials for `splits` key ranges: fp32 o [B*Hq*splits*D], then (m, l) pairs.
+size_t decode_partials_bytes(int B, int Hq, int D, int splits) {
+  const size_t rows = static_cast<size_t>(B) * Hq * splits;
+  const size_t po = (rows * D * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  return po + rows * sizeof(float2);
+}
+
 }  // namespace
 
 extern "C" {
@@ -461,5 +494,87 @@ RA_API int rope_attn_trace_read(void* host, size_t bytes) {
                                                                                       : RA_ERR_CUDA;
 }
 #endif
+
+ra_status rope_attn_decode_noalloc(const void* q, const void* k_cache_rot, const void* v_cache,
+                                   void* out, int B, int Hq, int Hkv, int Sk, int D,
+                                   float rope_base, int pos, int n_splits, ra_stream_t stream) {
+  if (!q || !k_cache_rot || !v_cache || !out) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache_rot) || !aligned16(v_cache) || !aligned16(out))
+    return RA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sk < 1 || D < 1 || pos < 0 || n_splits < 0)
+    return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const size_t qbytes = static_cast<size_t>(B) * Hq * D * 2;
+  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
+  if (overlap(out, qbytes, q, qbytes) || overlap(out, qbytes, k_cache_rot, kbytes) ||
+      overlap(out, qbytes, v_cache, kbytes))
+    return RA_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  const int hblocks = (G + 7) / 8;
+  if (static_cast<long long>(B) * Hkv * hblocks > 65535) return RA_ERR_UNSUPPORTED;
+  const int L = std::min(Sk, pos + 1);
+  // an explicit split count (as clamped by L) must fit the scratch; checked before any CUDA call
+  if (n_splits > 0) {
+    const int req = std::min(n_splits, std::max(1, (L + 63) / 64));
+    if (decode_partials_bytes(B, Hq, D, req) > kDecodeScratchBytes) {
+      std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                    "rope_attn_decode_noalloc: %zu bytes of partials exceed the %zu-byte scratch",
+                    decode_partials_bytes(B, Hq, D, req), kDecodeScratchBytes);
+      return RA_ERR_UNSUPPORTED;
+    }
+  }
+
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+  void* scratch = nullptr;
+  rs = decode_scratch(&scratch);
+  if (rs != RA_OK) return rs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  int splits = decode_splits(B, Hkv, G, L, ds->num_sms, n_splits);
+  // automatic choice: the largest count up to the usual one whose partials fit the scratch
+  while (splits > 1 && decode_partials_bytes(B, Hq, D, splits) > kDecodeScratchBytes) --splits;
+  const int chunk = ((L + splits - 1) / splits + 63) / 64 * 64;
+  splits = (L + chunk - 1) / chunk;
+  if (decode_partials_bytes(B, Hq, D, splits) > kDecodeScratchBytes) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "rope_attn_decode_noalloc: %zu bytes of partials exceed the %zu-byte scratch",
+                  decode_partials_bytes(B, Hq, D, splits), kDecodeScratchBytes);
+    return RA_ERR_UNSUPPORTED;
+  }
+  const size_t po_bytes =
+      (static_cast<size_t>(B) * Hq * splits * D * sizeof(float) + 255) & ~static_cast<size_t>(255);
+
+  CUtensorMap tk, tv;
+  rs = make_map(&tk, k_cache_rot, D, Sk, static_cast<long long>(B) * Hkv, 64);
+  if (rs == RA_OK) rs = make_map(&tv, v_cache, D, Sk, static_cast<long long>(B) * Hkv, 64);
+  if (rs != RA_OK) return rs;
+  ra::DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.part_o = static_cast<float*>(scratch);
+  p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(scratch) + po_bytes);
+  p.status = ds->status;
+  p.wait_limit = g_wait_limit.load();
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.Sk = Sk;
+  p.L = L;
+  p.pos = pos;
+  p.n_splits = splits;
+  p.chunk = chunk;
+  p.hblocks = hblocks;
+  p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+  p.rope_base = rope_base;
+  const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(B * Hkv * hblocks));
+  if (D == 64)
+    ra::decode_split_kernel<64><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
+  else
+    ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
+  ra::decode_combine_kernel<<<static_cast<unsigned>(B * Hq), D, 0, s>>>(
+      p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(out), splits, D);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "decode (no-alloc) launch");
+}
 
 }  // extern "C"
