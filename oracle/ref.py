@@ -38,6 +38,10 @@ Readings where the pages leave a step open (each also listed in the design notes
   every one of the D dimensions is rotated.
 * Decode: the single query at absolute position ``pos`` attends cache rows
   0..min(Sk, pos+1)-1, which hold keys that were already rotated when written.
+* Sliding window ("Building Self-Attention and Transformer Engines", §6.4 "Sliding Window
+  Attention (SWA) in Mistral 7B" and FAQ Q10: each token attends only to the nearest W
+  preceding tokens): a query at position p sees the keys at positions p-W+1 .. p, itself
+  included, so W = 1 attends only to itself; W = 0 means no window.
 """
 from __future__ import annotations
 
@@ -94,12 +98,15 @@ def _softmax_rows(s: np.ndarray) -> np.ndarray:
 
 
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool,
-              rows: np.ndarray | None = None, row_block: int = 1024) -> np.ndarray:
+              rows: np.ndarray | None = None, row_block: int = 1024,
+              window: int = 0) -> np.ndarray:
     """softmax(Q K^T / sqrt(D) + M) V with grouped KV heads, in float64.
 
     q: [B, Hq, Sq, D]; k, v: [B, Hkv, Sk, D] (no RoPE applied here).
     M is -inf where key j lies after query i under the bottom-right alignment
     (j > i + Sk - Sq), i.e. numpy's triu with offset Sk - Sq + 1; zero elsewhere.
+    With ``window`` W > 0, M is also -inf where key j lies W or more before the query
+    (j <= i + Sk - Sq - W).
     ``rows`` optionally selects which query rows to compute (each row of attention
     is independent of the others, so a subset is an exact check of those rows).
     The score block is materialised ``row_block`` rows at a time to bound memory.
@@ -125,12 +132,14 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool,
                 s = (q[b, h, r] @ k[b, kv].T) * scale            # [R, Sk]
                 if causal:
                     s = np.where(cols[None, :] > (r[:, None] + (Sk - Sq)), -np.inf, s)
+                if window > 0:
+                    s = np.where(cols[None, :] <= (r[:, None] + (Sk - Sq) - window), -np.inf, s)
                 out[b, h, r0:r0 + r.size] = _softmax_rows(s) @ v[b, kv]
     return out
 
 
 def rope_attn_fwd(q, k, v, rope_base: float, pos_offset: int = 0, causal: bool = True,
-                  rows=None) -> np.ndarray:
+                  rows=None, window: int = 0) -> np.ndarray:
     """The prefill result: rotate Q and K by their absolute positions, then attend.
 
     q: [B, Hq, Sq, D]; k, v: [B, Hkv, Sk, D]; inputs are widened to float64 first.
@@ -149,18 +158,21 @@ def rope_attn_fwd(q, k, v, rope_base: float, pos_offset: int = 0, causal: bool =
     else:
         q_rot = rope_rotate(q, qpos, rope_base)
     k_rot = rope_rotate(k, kpos, rope_base)
-    return attention(q_rot, k_rot, v, causal, rows=rows)
+    return attention(q_rot, k_rot, v, causal, rows=rows, window=window)
 
 
-def rope_attn_decode(q, k_cache_rot, v_cache, rope_base: float, pos: int) -> np.ndarray:
+def rope_attn_decode(q, k_cache_rot, v_cache, rope_base: float, pos: int,
+                     window: int = 0) -> np.ndarray:
     """One decode step: the query at absolute position ``pos`` (rotated here) attends
-    the first min(Sk, pos+1) rows of an already-rotated key cache.
+    the first min(Sk, pos+1) rows of an already-rotated key cache (with a window W > 0,
+    only the rows pos-W+1 .. pos of those).
 
     q: [B, Hq, 1, D]; k_cache_rot, v_cache: [B, Hkv, Sk, D]. Returns [B, Hq, 1, D].
     """
     q = np.asarray(q, dtype=np.float64)
     Sk = k_cache_rot.shape[2]
     L = min(Sk, pos + 1)
+    lo = max(0, pos - window + 1) if window > 0 else 0
     q_rot = rope_rotate(q, np.array([pos]), rope_base)
-    return attention(q_rot, np.asarray(k_cache_rot)[:, :, :L], np.asarray(v_cache)[:, :, :L],
+    return attention(q_rot, np.asarray(k_cache_rot)[:, :, lo:L], np.asarray(v_cache)[:, :, lo:L],
                      causal=False)

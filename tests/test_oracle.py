@@ -324,7 +324,83 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
     orig_attn = ref.attention
 
-    def no_mask(q, k, v, causal, rows=None, row_block=1024):
-        return orig_attn(q, k, v, False, rows, row_block)
+    def no_mask(q, k, v, causal, rows=None, row_block=1024, window=0):
+        return orig_attn(q, k, v, False, rows, row_block, window)
     monkeypatch.setattr(ref, "attention", no_mask)
     assert not causal_pin()
+    monkeypatch.setattr(ref, "attention", orig_attn)
+
+    def window_pin():
+        q, k, v = _rand((1, 1, 12, 4), 43), _rand((1, 1, 12, 4), 44), _rand((1, 1, 12, 4), 45)
+        return np.allclose(ref.rope_attn_fwd(q, k, v, 10000.0, window=1), v, atol=1e-14)
+
+    assert window_pin()
+
+    def window_off_by_one(q, k, v, causal, rows=None, row_block=1024, window=0):
+        return orig_attn(q, k, v, causal, rows, row_block, window + 1 if window else 0)
+    monkeypatch.setattr(ref, "attention", window_off_by_one)
+    assert not window_pin()
+
+
+# ----------------------------------------------------------------- sliding window
+
+def test_window_one_attends_only_itself():
+    # W = 1: each query sees only the key at its own position, so O[i] = V[i + Sk - Sq]
+    q, k, v = _rand((1, 2, 20, 8), 50), _rand((1, 2, 30, 8), 51), _rand((1, 2, 30, 8), 52)
+    o = oracle.rope_attn_fwd(q, k, v, 10000.0, causal=True, window=1)
+    np.testing.assert_allclose(o, v[:, :, 10:], atol=1e-14, rtol=0)
+
+
+def test_window_covering_everything_is_causal():
+    q, k, v = _rand((1, 2, 40, 8), 53), _rand((1, 2, 40, 8), 54), _rand((1, 2, 40, 8), 55)
+    np.testing.assert_allclose(oracle.rope_attn_fwd(q, k, v, 10000.0, window=40),
+                               oracle.rope_attn_fwd(q, k, v, 10000.0), atol=1e-14, rtol=0)
+
+
+def test_window_row_equals_causal_on_its_last_keys():
+    # row i with window W is plain attention of that query over keys i-W+1 .. i (RoPE is
+    # relative, so dropping the older keys and re-basing positions changes nothing)
+    S, W = 50, 7
+    q, k, v = _rand((1, 1, S, 8), 56), _rand((1, 1, S, 8), 57), _rand((1, 1, S, 8), 58)
+    o = oracle.rope_attn_fwd(q, k, v, 10000.0, window=W)
+    for i in (0, 3, 6, 7, 31, 49):
+        lo = max(0, i - W + 1)
+        sub = oracle.rope_attn_fwd(q[:, :, i:i + 1], k[:, :, lo:i + 1], v[:, :, lo:i + 1], 10000.0,
+                                   pos_offset=lo)
+        np.testing.assert_allclose(o[:, :, i], sub[:, :, 0], atol=1e-12, rtol=0)
+
+
+def test_window_decode_equals_last_prefill_row():
+    S, W = 45, 9
+    q, k, v = _rand((1, 4, S, 8), 59), _rand((1, 2, S, 8), 60), _rand((1, 2, S, 8), 61)
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0, window=W)
+    kc = oracle.rope_rotate(k, np.arange(S), 10000.0)
+    d = oracle.rope_attn_decode(q[:, :, S - 1:], kc, v, 10000.0, pos=S - 1, window=W)
+    np.testing.assert_allclose(d[:, :, 0], full[:, :, S - 1], atol=1e-13, rtol=0)
+
+
+def test_brute_force_window():
+    # scalar brute force with an explicit window test, written separately from the oracle
+    rng = np.random.default_rng(62)
+    Sq, Sk, W, D, off = 6, 9, 3, 4, 5
+    q, k, v = rng.standard_normal((1, 2, Sq, D)), rng.standard_normal((1, 1, Sk, D)), rng.standard_normal((1, 1, Sk, D))
+    want = np.zeros((1, 2, Sq, D))
+    for h in range(2):
+        for i in range(Sq):
+            pi = off + Sk - Sq + i
+            def rot(x, p):
+                out = np.zeros(D)
+                for t in range(D // 2):
+                    a = p * 10000.0 ** (-2.0 * t / D)
+                    out[2 * t] = x[2 * t] * math.cos(a) - x[2 * t + 1] * math.sin(a)
+                    out[2 * t + 1] = x[2 * t] * math.sin(a) + x[2 * t + 1] * math.cos(a)
+                return out
+            qi = rot(q[0, h, i], pi)
+            sc = [(j, float(qi @ rot(k[0, 0, j], off + j)) / math.sqrt(D)) for j in range(Sk)
+                  if pi - W < off + j <= pi]
+            mx = max(s for _, s in sc)
+            e = [(j, math.exp(s - mx)) for j, s in sc]
+            z = math.fsum(w for _, w in e)
+            want[0, h, i] = sum(w * v[0, 0, j] for j, w in e) / z
+    got = oracle.rope_attn_fwd(q, k, v, 10000.0, pos_offset=off, window=W)
+    np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
