@@ -129,6 +129,48 @@ __device__ __forceinline__ float softmax_p_store(const uint32_t* sr, float sl2, 
   return a0 + a1;
 }
 
+// Same as softmax_p_store, and also returns the max of the 128 raw scores in `mt` (eight
+// independent 3-input max chains interleaved with the exponentials, off the critical path).
+template <int kEmu>
+__device__ __forceinline__ float softmax_p_store_max(const uint32_t* sr, float sl2, float m,
+                                                     uint32_t tS, float& mt) {
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m, -m);
+  uint64_t acc2[4] = {0, 0, 0, 0};
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c2 = 0; c2 < 32; ++c2) {
+      const int c = h * 64 + 2 * c2;
+      const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
+      mx[c2 & 7] = max3f(mx[c2 & 7], s0, s1);
+      const uint64_t x2 = f2_fma(f2_pack(s0, s1), sl2x2, negm2);
+      uint64_t p2;
+      if ((c2 & 3) < kEmu) {
+        p2 = exp2_poly_x2(x2);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p2 = f2_pack(ex2(x0), ex2(x1));
+      }
+      acc2[c2 & 3] = f2_add(acc2[c2 & 3], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[c2] = pack_bf16(p0, p1);
+    }
+    tmem_st32(tS + 32 * h, pk);
+  }
+  mt = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+  const uint64_t a = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+  float a0, a1;
+  f2_unpack(a, a0, a1);
+  return a0 + a1;
+}
+
 #ifndef RA_EMU_PAIRS
 #define RA_EMU_PAIRS 0
 #endif
@@ -278,13 +320,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool ok = mbar_wait(bar(C::B_QREADY + 0), 0, lim, abort_flag, p.status) &&
                 mbar_wait(bar(C::B_FULL + kslot(0)), kpar(0), lim, abort_flag, p.status);
       if (ok) {
-        tc_fence_after();
         issue_s(0, kslot(0));
         umma_commit(bar(C::B_SFULL + 0));
         if (ns == 2) {
           ok = mbar_wait(bar(C::B_QREADY + 1), 0, lim, abort_flag, p.status);
           if (ok) {
-            tc_fence_after();
             issue_s(1, kslot(0));
             umma_commit(bar(C::B_SFULL + 1));
           }
@@ -305,7 +345,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (has_next) {
           if (!mbar_wait(bar(C::B_FULL + kslot(j + 1)), kpar(j + 1), lim, abort_flag, p.status))
             break;
-          tc_fence_after();
+          // (no tcgen05 fence: S reads only shared memory, synchronised by the mbarrier)
           RA_STAMP(3, j);
           issue_s(0, kslot(j + 1));
           RA_STAMP(4, j);
@@ -399,44 +439,58 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int c = 0; c < 128; ++c)
           if (c > lim_k) sr[c] = 0xff800000u;  // -inf
       }
-      // a7: online softmax with a lazily updated reference max
-      // tile max of the raw scores: eight independent 3-input max chains, then a tree
-      float mx[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        mx[k] = max3f(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]), __uint_as_float(sr[k + 16]));
-#pragma unroll
-      for (int c = 24; c < 120; c += 16)
+      // a7: online softmax with a lazily updated reference max m. Once a row has a
+      // reference, P is computed speculatively with it while the tile max is gathered
+      // on the side; only if some row's max grew by more than 8 (log2 units) does the warp
+      // redo the tile exactly (rescale O, P with the new reference). Either way every row
+      // ends with the same values as the plain max-first order.
+      float rs = 0.f;
+      bool done = false;
+      float mt = -INFINITY;
+      if (!__any_sync(0xffffffffu, m == -INFINITY)) {
+        rs = need_mask ? softmax_p_store_max<0>(sr, sl2, m, tS, mt)
+                       : softmax_p_store_max<kEmuPairs>(sr, sl2, m, tS, mt);
+        done = !__any_sync(0xffffffffu, fmaxf(m, mt * sl2) > m + 8.0f);
+      } else {
+        // tile max of the raw scores: eight independent 3-input max chains, then a tree
+        float mx[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mx[k] = max3f(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+          mx[k] = max3f(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]),
+                        __uint_as_float(sr[k + 16]));
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[120 + k]));
-      const float mt = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]),
-                             fmaxf(mx[6], mx[7]));
-      const float m_new = fmaxf(m, mt * sl2);
-      // Keep the old reference unless the max grew by more than 8 (P stays <= 256);
-      // O / l is exact for any common reference, so skipping the rescale is lossless.
-      const bool upd = m_new > m + 8.0f;
-      const float alpha = upd ? ex2(m - m_new) : 1.0f;
-      if (upd) m = m_new;
-      l *= alpha;
-      if (j > 0 && __any_sync(0xffffffffu, upd)) {
-        // a8: O_s *= alpha (PV_s(j-1) has completed: it was issued before S_s(j))
+        for (int c = 24; c < 120; c += 16)
 #pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + cb, o);
-          tmem_wait_ld();
+          for (int k = 0; k < 8; ++k)
+            mx[k] = max3f(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + cb, o);
-        }
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[120 + k]));
+        mt = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       }
-      // p = 2^(s * log2(e)/sqrt(D) - m) -> bf16 P over the S columns; unmasked tiles send
-      // part of the exponentials to the FMA pipe
-      const float rs = need_mask ? softmax_p_store<0>(sr, sl2, m, tS)
-                                 : softmax_p_store<kEmuPairs>(sr, sl2, m, tS);
+      if (!done) {
+        const float m_new = fmaxf(m, mt * sl2);
+        // Keep the old reference unless the max grew by more than 8 (P stays <= 256);
+        // O / l is exact for any common reference, so skipping the rescale is lossless.
+        const bool upd = m_new > m + 8.0f;
+        const float alpha = upd ? ex2(m - m_new) : 1.0f;
+        if (upd) m = m_new;
+        l *= alpha;
+        if (j > 0 && __any_sync(0xffffffffu, upd)) {
+          // a8: O_s *= alpha (PV_s(j-1) has completed: it was issued before S_s(j))
+#pragma unroll
+          for (int cb = 0; cb < D; cb += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + cb, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + cb, o);
+          }
+        }
+        // p = 2^(s * log2(e)/sqrt(D) - m) -> bf16 P over the S columns
+        rs = need_mask ? softmax_p_store<0>(sr, sl2, m, tS)
+                       : softmax_p_store<kEmuPairs>(sr, sl2, m, tS);
+      }
       l += rs;
       tmem_wait_st();
       tc_fence_before();
