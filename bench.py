@@ -43,9 +43,12 @@ from synthetic import DECODE, LLAMA, make_inputs  # noqa: E402
 PREFILL_W, DECODE_W = LLAMA, DECODE
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS, SPEC_HBM_GBS = 2250.0, 8000.0
-KERNEL_SOURCES = ["transformer_attention_04_b200/csrc/attn_fwd_sm100.cuh",
-                  "transformer_attention_04_b200/csrc/decode.cuh",
-                  "transformer_attention_04_b200/csrc/ptx.cuh"]
+KERNEL_SOURCES = {
+    "attn_fwd_sm100_kernel": ["transformer_attention_04_b200/csrc/attn_fwd_sm100.cuh",
+                              "transformer_attention_04_b200/csrc/ptx.cuh"],
+    "decode_split_kernel": ["transformer_attention_04_b200/csrc/decode.cuh",
+                            "transformer_attention_04_b200/csrc/ptx.cuh"],
+}
 
 
 def parse_args(argv=None):
@@ -57,6 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--profile-leg", choices=["prefill", "decode"], default=None,
+                    help="run only this leg, warm-up + steps launches, and print no JSON "
+                         "(the command that ncu captures wraps; holds only that leg's buffers)")
     a = ap.parse_args(argv)
     a.warmup = max(a.warmup, 3)
     return a
@@ -112,9 +118,10 @@ def measured_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel: str):
+    """sha256[:16] over the source files a kernel is compiled from."""
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -127,7 +134,7 @@ def recorded_traffic(kernel: str):
         with open(path) as f:
             d = json.load(f)
         e = d[kernel]
-        if e.get("source_hash") != kernel_source_hash():
+        if e.get("source_hash") != kernel_source_hash(kernel.split()[0]):
             return None
         return int(e["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
@@ -438,10 +445,34 @@ def e2e_leg(ra, args, world, dev, qp, kp, vp, qd, kd, vd):
             "steps": n}
 
 
+def run_profile_leg(args):
+    """One leg alone, for profiler captures: the same inputs and calls as the timed step."""
+    import transformer_attention_04_b200 as ra
+    dev = torch.device("cuda", 0)
+    if args.profile_leg == "prefill":
+        W = PREFILL_W
+        q, k, v = (t.to(dev) for t in make_inputs(W, rank_seed(0, 0)))
+        out = torch.empty_like(q)
+        call = lambda: ra.rope_attn_fwd(q, k, v, W.rope_base, 0, True, out=out)
+    else:
+        W = DECODE_W
+        q, k, v = (t.to(dev) for t in make_inputs(W, rank_seed(0, 1)))
+        out = torch.empty_like(q)
+        call = lambda: ra.rope_attn_decode(q, k, v, W.rope_base, W.decode_pos, out=out)
+    for _ in range(args.warmup + args.steps):
+        call()
+    torch.cuda.synchronize()
+    st = ra.rope_attn_get_device_status()
+    print(f"{args.profile_leg}: {args.warmup + args.steps} calls, device status {st}", flush=True)
+    return 0 if st == ra.RA_OK else 1
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_leg:
+        return run_profile_leg(args)
     return run_ours(args)
 
 
