@@ -6,4 +6,8 @@ from .ref import (  # noqa: F401
     query_positions,
     rope_attn_fwd,
     rope_attn_decode,
+    rope_attn_prefill_cached,
+    rope_attn_decode_step,
+    gather_pages,
+    rope_attn_decode_paged,
 )

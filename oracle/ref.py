@@ -54,6 +54,10 @@ __all__ = [
     "query_positions",
     "rope_attn_fwd",
     "rope_attn_decode",
+    "rope_attn_prefill_cached",
+    "rope_attn_decode_step",
+    "gather_pages",
+    "rope_attn_decode_paged",
 ]
 
 
@@ -176,3 +180,105 @@ def rope_attn_decode(q, k_cache_rot, v_cache, rope_base: float, pos: int,
     q_rot = rope_rotate(q, np.array([pos]), rope_base)
     return attention(q_rot, np.asarray(k_cache_rot)[:, :, lo:L], np.asarray(v_cache)[:, :, lo:L],
                      causal=False)
+
+
+# ----------------------------------------------------------------- KV-cache flow
+#
+# "Transformer internals: attention without the mysticism", "The KV cache and the memory
+# wall", and "Building Self-Attention and Transformer Engines" §6 (GQA & KV-cache
+# optimizations) with §6.2 (PagedAttention: the cache split into fixed 16-token blocks):
+# the keys and values of past tokens are kept and every new token reads them. Readings (also in the design notes): cache row j holds the key of absolute position
+# j, already rotated to that position; a prefill chunk of Sk new tokens starting at
+# position pos_offset is written to rows pos_offset .. pos_offset+Sk-1 and its queries attend
+# every cache row up to their own position; a decode step writes its new token at row pos[b]
+# and attends rows lo .. pos[b] of its own sequence.
+
+
+def rope_attn_prefill_cached(q, k_new, v_new, k_cache_rot, v_cache, rope_base: float,
+                             pos_offset: int, causal: bool = True, window: int = 0):
+    """Chunked prefill into a KV cache. Returns (out, k_cache_rot', v_cache').
+
+    q: [B, Hq, Sq, D]; k_new, v_new: [B, Hkv, Sk, D] (keys not rotated);
+    k_cache_rot, v_cache: [B, Hkv, S_cache, D] whose rows 0..pos_offset-1 hold the earlier
+    context (keys rotated). The chunk's keys are rotated to positions pos_offset + j and
+    stored with the values at rows pos_offset + j; the Sq queries sit at positions
+    pos_offset + Sk - Sq + i and attend the T = pos_offset + Sk cache rows under the mask.
+    """
+    k_new = np.asarray(k_new, dtype=np.float64)
+    Sk = k_new.shape[2]
+    kc = np.array(k_cache_rot, dtype=np.float64, copy=True)
+    vc = np.array(v_cache, dtype=np.float64, copy=True)
+    T = pos_offset + Sk
+    if T > kc.shape[2]:
+        raise ValueError("chunk does not fit the cache")
+    kc[:, :, pos_offset:T] = rope_rotate(k_new, pos_offset + np.arange(Sk), rope_base)
+    vc[:, :, pos_offset:T] = np.asarray(v_new, dtype=np.float64)
+    q = np.asarray(q, dtype=np.float64)
+    Sq = q.shape[2]
+    q_rot = rope_rotate(q, query_positions(Sq, T, 0), rope_base)
+    out = attention(q_rot, kc[:, :, :T], vc[:, :, :T], causal, window=window)
+    return out, kc, vc
+
+
+def rope_attn_decode_step(q, k_new, v_new, k_cache_rot, v_cache, rope_base: float, pos,
+                          window: int = 0):
+    """One decode step of a batch whose sequences sit at their own positions pos[b].
+
+    q: [B, Hq, 1, D]; k_new, v_new: [B, Hkv, 1, D] (the new token's key, not rotated, and
+    value), or None to attend the cache as it is; caches [B, Hkv, S_cache, D].
+    The new key is rotated to pos[b] and stored with the value at row pos[b]; the query,
+    rotated to pos[b], attends rows lo .. pos[b] (lo = pos[b]-W+1 with a window W, else 0).
+    Returns (out [B, Hq, 1, D], k_cache_rot', v_cache').
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kc = np.array(k_cache_rot, dtype=np.float64, copy=True)
+    vc = np.array(v_cache, dtype=np.float64, copy=True)
+    B = q.shape[0]
+    out = np.empty(q.shape, dtype=np.float64)
+    for b in range(B):
+        p = int(pos[b])
+        if k_new is not None:
+            kc[b, :, p] = rope_rotate(np.asarray(k_new, dtype=np.float64)[b, :, 0:1],
+                                      np.array([p]), rope_base)[:, 0]
+            vc[b, :, p] = np.asarray(v_new, dtype=np.float64)[b, :, 0]
+        out[b:b + 1] = rope_attn_decode(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], rope_base, p,
+                                        window=window)
+    return out, kc, vc
+
+
+def gather_pages(pool, block_table, b: int, n_rows: int):
+    """Rows 0..n_rows-1 of sequence b from a paged pool [num_blocks, Hkv, page, D]:
+    row j lives in block block_table[b, j // page] at offset j % page ("Building
+    Self-Attention and Transformer Engines" §6.2 PagedAttention: a sequence's cache is a
+    list of fixed-size physical blocks). Returns [Hkv, n_rows, D]."""
+    pool = np.asarray(pool)
+    page = pool.shape[2]
+    rows = [pool[int(block_table[b, j // page]), :, j % page] for j in range(n_rows)]
+    return np.stack(rows, axis=1) if rows else np.zeros((pool.shape[1], 0, pool.shape[3]))
+
+
+def rope_attn_decode_paged(q, k_new, v_new, k_pool_rot, v_pool, block_table, rope_base: float,
+                           pos, window: int = 0):
+    """rope_attn_decode_step over a paged cache. Returns (out, k_pool', v_pool').
+
+    The new token (if given) is written to the pool slot of row pos[b]; then each
+    sequence's rows 0..pos[b] are gathered through its block table and attended as in the
+    contiguous step.
+    """
+    kp = np.array(k_pool_rot, dtype=np.float64, copy=True)
+    vp = np.array(v_pool, dtype=np.float64, copy=True)
+    page = kp.shape[2]
+    q = np.asarray(q, dtype=np.float64)
+    B = q.shape[0]
+    out = np.empty(q.shape, dtype=np.float64)
+    for b in range(B):
+        p = int(pos[b])
+        blk, off = int(block_table[b, p // page]), p % page
+        if k_new is not None:
+            kp[blk, :, off] = rope_rotate(np.asarray(k_new, dtype=np.float64)[b, :, 0:1],
+                                          np.array([p]), rope_base)[:, 0]
+            vp[blk, :, off] = np.asarray(v_new, dtype=np.float64)[b, :, 0]
+        kc = gather_pages(kp, block_table, b, p + 1)[None]
+        vc = gather_pages(vp, block_table, b, p + 1)[None]
+        out[b:b + 1] = rope_attn_decode(q[b:b + 1], kc, vc, rope_base, p, window=window)
+    return out, kp, vp

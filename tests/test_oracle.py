@@ -404,3 +404,96 @@ def test_brute_force_window():
             want[0, h, i] = sum(w * v[0, 0, j] for j, w in e) / z
     got = oracle.rope_attn_fwd(q, k, v, 10000.0, pos_offset=off, window=W)
     np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
+
+
+# ----------------------------------------------------------------- KV-cache flow
+
+def _kv_seq(seed, B=2, Hq=4, Hkv=2, S=40, D=8):
+    r = np.random.default_rng(seed)
+    return (r.standard_normal((B, Hq, S, D)), r.standard_normal((B, Hkv, S, D)),
+            r.standard_normal((B, Hkv, S, D)))
+
+
+@pytest.mark.parametrize("P,window", [(0, 0), (17, 0), (25, 9), (39, 0)])
+def test_chunked_prefill_equals_full_prefill(P, window):
+    # prefilling tokens P.. on top of a cache that holds tokens 0..P-1 gives the same rows as
+    # one prefill of the whole sequence (and the cache ends up holding all rotated keys)
+    q, k, v = _kv_seq(70)
+    S, cap = k.shape[2], 48
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0, window=window)
+    kc = np.full((2, 2, cap, 8), np.nan)
+    vc = np.full((2, 2, cap, 8), np.nan)
+    kc[:, :, :P] = oracle.rope_rotate(k[:, :, :P], np.arange(P), 10000.0)
+    vc[:, :, :P] = v[:, :, :P]
+    out, kc2, vc2 = oracle.rope_attn_prefill_cached(q[:, :, P:], k[:, :, P:], v[:, :, P:], kc, vc,
+                                                    10000.0, P, window=window)
+    np.testing.assert_allclose(out, full[:, :, P:], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(kc2[:, :, :S], oracle.rope_rotate(k, np.arange(S), 10000.0),
+                               atol=1e-14, rtol=0)
+    np.testing.assert_array_equal(vc2[:, :, :S], v)
+    assert np.isnan(kc2[:, :, S:]).all() and np.isnan(vc2[:, :, S:]).all()  # rows past T untouched
+
+
+def test_token_by_token_decode_equals_prefill():
+    # decoding the sequence one token at a time from an empty cache (each step appends its
+    # own key/value at pos) reproduces every row of the causal prefill
+    q, k, v = _kv_seq(71, S=24)
+    S = k.shape[2]
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0)
+    kc = np.full((2, 2, 32, 8), np.nan)
+    vc = np.full((2, 2, 32, 8), np.nan)
+    for p in range(S):
+        out, kc, vc = oracle.rope_attn_decode_step(q[:, :, p:p + 1], k[:, :, p:p + 1],
+                                                   v[:, :, p:p + 1], kc, vc, 10000.0, [p, p])
+        np.testing.assert_allclose(out[:, :, 0], full[:, :, p], atol=1e-12, rtol=0)
+
+
+def test_varlen_decode_each_sequence_at_its_position():
+    q, k, v = _kv_seq(72, B=3, S=30)
+    pos = [29, 4, 17]
+    kc = oracle.rope_rotate(k, np.arange(30), 10000.0)
+    vc = v.copy()
+    for window in (0, 6):
+        full = oracle.rope_attn_fwd(q, k, v, 10000.0, window=window)
+        qd = np.stack([q[b, :, pos[b]] for b in range(3)])[:, :, None]
+        # the new tokens are the keys already at pos[b]: appending them again is a no-op
+        kn = np.stack([k[b, :, pos[b]] for b in range(3)])[:, :, None]
+        vn = np.stack([v[b, :, pos[b]] for b in range(3)])[:, :, None]
+        out, kc2, vc2 = oracle.rope_attn_decode_step(qd, kn, vn, kc, vc, 10000.0, pos, window)
+        for b in range(3):
+            np.testing.assert_allclose(out[b, :, 0], full[b, :, pos[b]], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(kc2, kc, atol=1e-14, rtol=0)
+
+
+def test_gather_pages_by_hand():
+    # page 2, blocks [3, 0, 2]: rows 0..5 are block 3 rows 0,1, block 0 rows 0,1, block 2 rows 0,1
+    pool = np.zeros((4, 1, 2, 1))
+    for blk in range(4):
+        for off in range(2):
+            pool[blk, 0, off, 0] = 100 * blk + off
+    g = oracle.gather_pages(pool, np.array([[3, 0, 2]]), 0, 6)
+    assert g[0, :, 0].tolist() == [300, 301, 0, 1, 200, 201]
+
+
+def test_paged_decode_equals_contiguous():
+    rng = np.random.default_rng(73)
+    B, Hq, Hkv, D, page, nblk = 3, 4, 2, 8, 4, 9
+    pos = [10, 3, 7]
+    q = rng.standard_normal((B, Hq, 1, D))
+    kn, vn = rng.standard_normal((B, Hkv, 1, D)), rng.standard_normal((B, Hkv, 1, D))
+    kc, vc = rng.standard_normal((B, Hkv, 12, D)), rng.standard_normal((B, Hkv, 12, D))
+    # scatter each sequence's 12 rows over 3 pages of a shuffled pool
+    perm = rng.permutation(nblk)
+    table = perm.reshape(B, 3)
+    kp = np.full((nblk, Hkv, page, D), np.nan)
+    vp = np.full((nblk, Hkv, page, D), np.nan)
+    for b in range(B):
+        for j in range(12):
+            kp[table[b, j // page], :, j % page] = kc[b, :, j]
+            vp[table[b, j // page], :, j % page] = vc[b, :, j]
+    for window in (0, 5):
+        want, kc2, _ = oracle.rope_attn_decode_step(q, kn, vn, kc, vc, 10000.0, pos, window)
+        got, kp2, _ = oracle.rope_attn_decode_paged(q, kn, vn, kp, vp, table, 10000.0, pos, window)
+        np.testing.assert_array_equal(got, want)
+        for b in range(B):
+            np.testing.assert_array_equal(oracle.gather_pages(kp2, table, b, 12), kc2[b])
