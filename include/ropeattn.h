@@ -70,6 +70,32 @@ RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void
                         int causal, ra_stream_t stream);
 
 /*
+ * Prefill with a sliding window and/or straight into a KV cache (chunked prefill).
+ *
+ * window W > 0 (causal only): key j is visible to query row i iff
+ *   p_q(i) - W < p_k(j) <= p_q(i), i.e. each token sees its nearest W tokens, itself included
+ * ("Building Self-Attention and Transformer Engines" (codingpancake.com), §6.4 "Sliding
+ * Window Attention (SWA) in Mistral 7B" and FAQ Q10). W = 0: no window. KV tiles wholly
+ * outside every row's window are skipped.
+ *
+ * k_cache_rot == v_cache == NULL: the same attention as rope_attn_fwd (S_cache ignored).
+ * Otherwise the two caches [B, Hkv, S_cache, D] bf16 (read and written) hold the context:
+ * rows 0 .. pos_offset-1 carry the earlier tokens' rotated keys and values. The call rotates
+ * the chunk's keys k [B, Hkv, Sk, D] to positions pos_offset + j and stores them, and v,
+ * at rows pos_offset + j (j < Sk); then the Sq queries, at positions
+ * pos_offset + Sk - Sq + i, attend all T = pos_offset + Sk cache rows under the mask. With
+ * pos_offset = 0 the result equals rope_attn_fwd and the caches are ready for
+ * rope_attn_decode / rope_attn_decode_step ("Transformer internals: attention without the
+ * mysticism", "The KV cache and the memory wall"). Cache rows >= T are neither read nor
+ * written. Requires T <= S_cache, causal => Sq <= T; the caches must not overlap q, k, v,
+ * out or each other. Other arguments and errors as rope_attn_fwd.
+ */
+RA_API ra_status rope_attn_prefill(const void* q, const void* k, const void* v, void* out,
+                                   void* k_cache_rot, void* v_cache, int S_cache, int B, int Hq,
+                                   int Hkv, int Sq, int Sk, int D, float rope_base,
+                                   int pos_offset, int causal, int window, ra_stream_t stream);
+
+/*
  * RoPE rotation of a whole tensor (builds a pre-rotated key cache for rope_attn_decode).
  *
  *   x_rot[b,h,s,2i]   = x[b,h,s,2i] cos(m theta_i) - x[b,h,s,2i+1] sin(m theta_i)
@@ -129,13 +155,63 @@ RA_API ra_status rope_attn_decode_noalloc(const void* q, const void* k_cache_rot
                                           int Sk, int D, float rope_base, int pos, int n_splits,
                                           ra_stream_t stream);
 
+/*
+ * One decode step of a batch whose sequences sit at their own positions, with the step's
+ * new token appended to the cache inside the call (varlen batch).
+ *
+ *   pos [B] int32, DEVICE memory: sequence b's new token is at absolute position pos[b]
+ *   (cache rows 0 .. pos[b]-1 hold its earlier tokens, keys rotated).
+ *   k_new, v_new [B, Hkv, 1, D] bf16 (keys NOT rotated), or both NULL to attend the cache
+ *   as it is (row pos[b] must then already hold the token).
+ *   k_cache_rot, v_cache [B, Hkv, S_cache, D] bf16: with k_new, row pos[b] of each is
+ *   overwritten with R(pos[b]) k_new and v_new before it is read; no other row is written.
+ *   out[b,h,0,:] = sum_{lo<=j<=pos[b]} softmax_j(<R(pos[b]) q[b,h,0,:], k[b,h/G,j,:]>/sqrt(D))
+ *                  * v[b,h/G,j,:],   lo = max(0, pos[b]-W+1) with window W > 0, else 0.
+ *   max_pos: an upper bound on every pos[b], 0 <= max_pos < S_cache; the launch is sized
+ *   for it (fewer rows, fewer CTAs). A pos[b] outside [0, max_pos] is found by the kernel:
+ *   that sequence is not computed and rope_attn_get_device_status() returns
+ *   RA_ERR_INVALID_ARG.
+ * KV-cache decode of "Transformer internals: attention without the mysticism" ("The KV
+ * cache and the memory wall"); window as in rope_attn_prefill. The caches must not overlap
+ * q, k_new, v_new, out or each other. Other arguments and errors as rope_attn_decode.
+ */
+RA_API ra_status rope_attn_decode_step(const void* q, const void* k_new, const void* v_new,
+                                       void* k_cache_rot, void* v_cache, void* out,
+                                       const int* pos, int B, int Hq, int Hkv, int S_cache, int D,
+                                       float rope_base, int max_pos, int window, int n_splits,
+                                       ra_stream_t stream);
+
+/*
+ * rope_attn_decode_step over a paged cache ("Building Self-Attention and Transformer
+ * Engines" (codingpancake.com), §6.2 "PagedAttention": the cache is cut into fixed-size
+ * physical blocks, 16 tokens each there, that a sequence reaches through its block table).
+ *
+ *   k_pool_rot, v_pool [num_blocks, Hkv, page_size, D] bf16: block n holds page_size
+ *   consecutive rows of one sequence for every KV head.
+ *   block_table [B, max_blocks_per_seq] int32, DEVICE memory: row j of sequence b is row
+ *   j % page_size of block block_table[b][j / page_size].
+ *   page_size in {8, 16, 32, 64}; every pos[b] <= max_pos < max_blocks_per_seq * page_size.
+ * Entries for the pages of rows lo .. pos[b] must name blocks in [0, num_blocks); an entry
+ * out of range reads as zeros, and for the page receiving the appended token it is reported
+ * as RA_ERR_INVALID_ARG by rope_attn_get_device_status() (nothing is written then). Entries
+ * of other pages are never dereferenced. Everything else as rope_attn_decode_step.
+ */
+RA_API ra_status rope_attn_decode_paged(const void* q, const void* k_new, const void* v_new,
+                                        void* k_pool_rot, void* v_pool, const int* block_table,
+                                        void* out, const int* pos, int B, int Hq, int Hkv, int D,
+                                        int page_size, int max_blocks_per_seq, int num_blocks,
+                                        float rope_base, int max_pos, int window, int n_splits,
+                                        ra_stream_t stream);
+
 /* Split count rope_attn_decode uses for these sizes when n_splits == 0. */
 RA_API int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos);
 
 /*
  * Synchronises `stream`, returns the sticky device status of the current device and clears
- * it: RA_OK, RA_ERR_DEVICE_TIMEOUT, or RA_ERR_CUDA if the sync failed or a kernel found its
- * shared-memory base misaligned (it then did no work; see rope_attn_last_cuda_error).
+ * it: RA_OK, RA_ERR_DEVICE_TIMEOUT, RA_ERR_INVALID_ARG if a kernel found a per-sequence
+ * position or block-table entry out of range, or RA_ERR_CUDA if the sync failed or a kernel
+ * found its shared-memory base misaligned (it then did no work; see
+ * rope_attn_last_cuda_error).
  */
 RA_API ra_status rope_attn_get_device_status(ra_stream_t stream);
 

@@ -15,8 +15,11 @@ from ._lib import (  # noqa: F401
     rope_attn_decode,
     rope_attn_decode_auto_splits,
     rope_attn_decode_noalloc,
+    rope_attn_decode_paged,
+    rope_attn_decode_step,
     rope_attn_fwd,
     rope_attn_get_device_status,
+    rope_attn_prefill,
     rope_attn_profile_enable,
     rope_attn_profile_read,
     rope_attn_rotate,

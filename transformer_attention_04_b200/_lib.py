@@ -21,9 +21,15 @@ RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_DEVICE_TIMEOU
 _P, _I, _F, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
 SIGNATURES = {
     "rope_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "rope_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
+                               _P]),
     "rope_attn_rotate": (_I, [_P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "rope_attn_decode": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "rope_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "rope_attn_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I,
+                                   _I, _P]),
+    "rope_attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                    _F, _I, _I, _I, _P]),
     "rope_attn_decode_auto_splits": (_I, [_I, _I, _I, _I, _I, _I]),
     "rope_attn_get_device_status": (_I, [_P]),
     "rope_attn_set_wait_limit": (_LL, [_LL]),
@@ -98,6 +104,112 @@ def rope_attn_fwd(q, k, v, rope_base: float, pos_offset: int = 0, causal: bool =
                              Sq, Sk, D, float(rope_base), int(pos_offset), int(bool(causal)),
                              _stream(stream))
     _raise(st, "rope_attn_fwd")
+    return out
+
+
+def rope_attn_prefill(q, k, v, rope_base: float, pos_offset: int = 0, causal: bool = True,
+                      window: int = 0, k_cache_rot=None, v_cache=None, out=None, stream=None):
+    """Prefill with an optional sliding window, optionally into a KV cache (chunked prefill).
+
+    q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D]. With caches [B,Hkv,S_cache,D] the chunk's rotated keys
+    and values go to rows pos_offset.. and the queries attend all pos_offset+Sk cache rows.
+    """
+    _check(q, "q")
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, S, D]")
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    _check(k, "k", (B, Hkv, Sk, D))
+    _check(v, "v", (B, Hkv, Sk, D))
+    S_cache, kc, vc = 0, 0, 0
+    if (k_cache_rot is None) != (v_cache is None):
+        raise ValueError("give both caches or neither")
+    if k_cache_rot is not None:
+        S_cache = k_cache_rot.shape[2]
+        _check(k_cache_rot, "k_cache_rot", (B, Hkv, S_cache, D))
+        _check(v_cache, "v_cache", (B, Hkv, S_cache, D))
+        kc, vc = k_cache_rot.data_ptr(), v_cache.data_ptr()
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    st = lib().rope_attn_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), kc, vc,
+                                 S_cache, B, Hq, Hkv, Sq, Sk, D, float(rope_base), int(pos_offset),
+                                 int(bool(causal)), int(window), _stream(stream))
+    _raise(st, "rope_attn_prefill")
+    return out
+
+
+def _check_pos(pos, B):
+    if not isinstance(pos, torch.Tensor) or not pos.is_cuda or pos.dtype != torch.int32:
+        raise ValueError("pos must be an int32 CUDA tensor")
+    if tuple(pos.shape) != (B,) or not pos.is_contiguous():
+        raise ValueError(f"pos must have shape ({B},)")
+
+
+def rope_attn_decode_step(q, k_cache_rot, v_cache, pos, max_pos: int, rope_base: float,
+                          k_new=None, v_new=None, window: int = 0, n_splits: int = 0, out=None,
+                          stream=None):
+    """Decode step at per-sequence positions pos [B] (int32, device), appending the new token
+    (k_new/v_new [B,Hkv,1,D], keys not rotated) to the caches [B,Hkv,S_cache,D] at row pos[b]."""
+    _check(q, "q")
+    B, Hq, one, D = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query row per head")
+    Hkv, S_cache = k_cache_rot.shape[1], k_cache_rot.shape[2]
+    _check(k_cache_rot, "k_cache_rot", (B, Hkv, S_cache, D))
+    _check(v_cache, "v_cache", (B, Hkv, S_cache, D))
+    _check_pos(pos, B)
+    kn = vn = 0
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new or neither")
+    if k_new is not None:
+        _check(k_new, "k_new", (B, Hkv, 1, D))
+        _check(v_new, "v_new", (B, Hkv, 1, D))
+        kn, vn = k_new.data_ptr(), v_new.data_ptr()
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    st = lib().rope_attn_decode_step(q.data_ptr(), kn, vn, k_cache_rot.data_ptr(),
+                                     v_cache.data_ptr(), out.data_ptr(), pos.data_ptr(), B, Hq, Hkv,
+                                     S_cache, D, float(rope_base), int(max_pos), int(window),
+                                     int(n_splits), _stream(stream))
+    _raise(st, "rope_attn_decode_step")
+    return out
+
+
+def rope_attn_decode_paged(q, k_pool_rot, v_pool, block_table, pos, max_pos: int,
+                           rope_base: float, k_new=None, v_new=None, window: int = 0,
+                           n_splits: int = 0, out=None, stream=None):
+    """rope_attn_decode_step over a paged pool [num_blocks,Hkv,page,D] and a block table
+    [B, max_blocks] (int32, device)."""
+    _check(q, "q")
+    B, Hq, one, D = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query row per head")
+    nb, Hkv, page = k_pool_rot.shape[0], k_pool_rot.shape[1], k_pool_rot.shape[2]
+    _check(k_pool_rot, "k_pool_rot", (nb, Hkv, page, D))
+    _check(v_pool, "v_pool", (nb, Hkv, page, D))
+    _check_pos(pos, B)
+    if (not isinstance(block_table, torch.Tensor) or not block_table.is_cuda or
+            block_table.dtype != torch.int32 or block_table.dim() != 2 or
+            block_table.shape[0] != B or not block_table.is_contiguous()):
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor [B, max_blocks]")
+    kn = vn = 0
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new or neither")
+    if k_new is not None:
+        _check(k_new, "k_new", (B, Hkv, 1, D))
+        _check(v_new, "v_new", (B, Hkv, 1, D))
+        kn, vn = k_new.data_ptr(), v_new.data_ptr()
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", q.shape)
+    st = lib().rope_attn_decode_paged(q.data_ptr(), kn, vn, k_pool_rot.data_ptr(),
+                                      v_pool.data_ptr(), block_table.data_ptr(), out.data_ptr(),
+                                      pos.data_ptr(), B, Hq, Hkv, D, page, block_table.shape[1], nb,
+                                      float(rope_base), int(max_pos), int(window), int(n_splits),
+                                      _stream(stream))
+    _raise(st, "rope_attn_decode_paged")
     return out
 
 

@@ -62,6 +62,7 @@ struct FwdParams {
   int ppg;              // CTA units per (batch, KV group, query tile) = G / n_slots
   int n_qtiles;         // ceil(Sq / 128)
   int causal;
+  int window;           // 0 = none; else key j is allowed to query row i iff j > i + Sk - Sq - window
   int q_tab_off;        // table row of query row 0
   float scale_log2;     // log2(e) / sqrt(D)
 };
@@ -211,6 +212,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int off = p.Sk - p.Sq;  // query row i sits at key index i + off
   int n_kv = (p.Sk + 127) / 128;
   if (p.causal) n_kv = min(n_kv, (min(p.Sq - 1, q0 + 127) + off) / 128 + 1);
+  // a6 with a sliding window: tiles wholly below the first row's window are skipped too
+  const int j_lo = (p.window > 0) ? max(0, q0 + off - p.window + 1) / 128 : 0;
+  const int n_it = n_kv - j_lo;  // KV tiles this CTA visits: j_lo .. n_kv - 1
   const int ns = p.n_slots;
 
   if (threadIdx.x == 0) {
@@ -263,7 +267,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       // ring item i: tile i/2 of K (i even) or V (i odd), in slot i % NSLOT
       int issued = 0;
-      for (int i = 0; i < 2 * n_kv; ++i) {
+      for (int i = 0; i < 2 * n_it; ++i) {
         const int sl = i % C::NSLOT;
         if (!(i & 1)) RA_STAMP(14, i >> 1);
         if (i >= C::NSLOT && !mbar_wait(bar(C::B_EMPTY + sl), ((i / C::NSLOT) - 1) & 1,
@@ -273,7 +277,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_expect_tx(bar(C::B_FULL + sl), C::TILE);
         const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_3d_hint(sRing + sl * C::TILE + kb * C::BLK, map, kb * 64, (i >> 1) * 128, kv_bh,
+          tma_load_3d_hint(sRing + sl * C::TILE + kb * C::BLK, map, kb * 64, (j_lo + (i >> 1)) * 128, kv_bh,
                            bar(C::B_FULL + sl), pol_keep);
         issued = i + 1;
       }
@@ -331,8 +335,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         umma_commit(bar(C::B_EMPTY + kslot(0)));
       }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const bool has_next = j + 1 < n_kv;
+      for (int j = 0; ok && j < n_it; ++j) {  // j counts visited tiles
+        const bool has_next = j + 1 < n_it;
         RA_STAMP(0, j);
         if (!mbar_wait(bar(C::B_PFULL + 0), j & 1, lim, abort_flag, p.status) ||
             !mbar_wait(bar(C::B_FULL + vslot(j)), vpar(j), lim, abort_flag, p.status))
@@ -416,7 +420,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     float l = 0.f;        // running row sum of 2^(x - m)
     const float sl2 = p.scale_log2;
     const int lim_causal = min(p.Sk - 1, qrow + off);
-    for (int j = 0; ok && j < n_kv; ++j) {
+    for (int j = 0; ok && j < n_it; ++j) {  // j counts visited tiles; KV tile j_lo + j
       if (!mbar_wait_warp(bar(C::B_SFULL + s), j & 1, lim, abort_flag, p.status)) {
         ok = false;
         break;
@@ -431,13 +435,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_wait_ld();
 
       // a6: causal / sequence-end mask, only on tiles that reach past some row's limit
-      const int kbase = j * 128;
-      const bool need_mask = (kbase + 128 > p.Sk) || (p.causal && kbase + 127 > q0 + off);
+      const int kbase = (j_lo + j) * 128;
+      const bool need_mask = (kbase + 128 > p.Sk) || (p.causal && kbase + 127 > q0 + off) ||
+                             (p.window > 0 && kbase + p.window < q0 + 128 + off);
       if (need_mask) {
         const int lim_k = (p.causal ? lim_causal : p.Sk - 1) - kbase;
+        const int lo_k = (p.window > 0) ? qrow + off - p.window + 1 - kbase : 0;
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (c > lim_k) sr[c] = 0xff800000u;  // -inf
+          if (c > lim_k || c < lo_k) sr[c] = 0xff800000u;  // -inf
       }
       // a7: online softmax with a lazily updated reference max m. Once a row has a
       // reference, P is computed speculatively with it while the tile max is gathered
@@ -487,9 +493,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_st32(tO + cb, o);
           }
         }
-        // p = 2^(s * log2(e)/sqrt(D) - m) -> bf16 P over the S columns
-        rs = need_mask ? softmax_p_store<0>(sr, sl2, m, tS)
-                       : softmax_p_store<kEmuPairs>(sr, sl2, m, tS);
+        // p = 2^(s * log2(e)/sqrt(D) - m) -> bf16 P over the S columns; a row that has seen
+        // no allowed key yet (only under a window) keeps m = -inf and gets P = 0
+        const float m_use = (m == -INFINITY) ? 0.f : m;
+        rs = need_mask ? softmax_p_store<0>(sr, sl2, m_use, tS)
+                       : softmax_p_store<kEmuPairs>(sr, sl2, m_use, tS);
       }
       l += rs;
       tmem_wait_st();

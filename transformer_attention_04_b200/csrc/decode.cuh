@@ -18,6 +18,20 @@
 // merged in shared memory, and the CTA writes one unnormalised partial (o, m, l) per head.
 // decode_combine_kernel then merges the splits:
 //   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+//
+// The same kernel serves every decode entry:
+// * sequences at their own positions pos[b] (a varlen batch), each attending rows
+//   lo_b .. pos_b with lo_b = pos_b - W + 1 under a sliding window W ("Building
+//   Self-Attention and Transformer Engines" §6.4), else 0;
+// * an optional append of the step's new token: the CTA whose key range holds row pos_b
+//   rotates the new key to pos_b, stores it and the new value into the cache, and only then
+//   loads its tiles, so the step attends its own token;
+// * a contiguous cache [B, Hkv, S_cache, D] or a paged pool [num_blocks, Hkv, page, D]
+//   reached through a block table (§6.2 PagedAttention), one TMA box per page.
+// Key ranges are cut on 64-row boundaries of the absolute row index, so a tile is always
+// whole pages. Rows of an edge tile outside [lo_b, L_b) are masked in S and their V rows
+// are zeroed in shared memory before the PV product, so whatever those rows hold (stale
+// cache contents, another sequence's page) cannot leak in, not even as NaN * 0.
 #pragma once
 
 #include "ptx.cuh"
@@ -31,14 +45,28 @@ struct DecParams {
   float2* part_ml;         // [B * Hq, n_splits] (m, l), m in log2 units of the scaled score
   unsigned int* status;
   long long wait_limit;
-  int B, Hq, Hkv, G, Sk;
-  int L;          // keys attended: min(Sk, pos + 1)
-  int pos;        // absolute position of the query
+  int B, Hq, Hkv, G;
+  int cap;        // rows one sequence can hold: S_cache, or max_blocks * page
+  int pos;        // position of every sequence when pos_arr is null
+  const int* pos_arr;  // [B] per-sequence positions (device memory), or null
+  int max_pos;    // bound on the positions the launch was sized for (checked)
+  int window;     // 0 = no window; else keys pos-W+1 .. pos
   int n_splits;   // splits actually launched
   int chunk;      // keys per split (multiple of 64)
   int hblocks;    // ceil(G / 8): blocks of 8 query heads per KV head
   float scale_log2;
   float rope_base;
+  // paged pool (page == 0: contiguous cache, maps over [B * Hkv, S_cache, D])
+  int page;                // rows per page (divides 64)
+  const int* block_table;  // [B, max_blocks]
+  int max_blocks;
+  int num_blocks;          // blocks in the pool (table entries are checked against it)
+  // append of the step's token (k_new == null: none)
+  const __nv_bfloat16* k_new;  // [B, Hkv, 1, D], not rotated
+  const __nv_bfloat16* v_new;  // [B, Hkv, 1, D]
+  __nv_bfloat16* k_cache;      // the memory tm_k covers
+  __nv_bfloat16* v_cache;      // the memory tm_v covers
+  int S_cache;
 };
 
 template <int D>
@@ -90,9 +118,21 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   const int hb = blockIdx.y % p.hblocks;
   const int kv_bh = blockIdx.y / p.hblocks;  // b * Hkv + kv head
   const int b = kv_bh / p.Hkv, g = kv_bh % p.Hkv;
-  const int kstart = split * p.chunk;
-  const int kend = min(p.L, kstart + p.chunk);
-  const int n_tiles = kend > kstart ? (kend - kstart + C::TK - 1) / C::TK : 0;
+  // this sequence's rows lo .. L-1; the launch covers rows (lo & ~63) + [0, n_splits * chunk)
+  const int pos_b = p.pos_arr ? p.pos_arr[b] : p.pos;
+  const int lo = (p.window > 0) ? max(0, pos_b - p.window + 1) : 0;
+  const int L0 = min(p.cap, pos_b + 1);
+  // (only the scalar-position contiguous call may name a position past the cache's end:
+  // it then attends the whole cache)
+  const bool strict = p.pos_arr != nullptr || p.page != 0 || p.k_new != nullptr;
+  const bool bad = pos_b < 0 || pos_b > p.max_pos || (strict && pos_b >= p.cap) ||
+                   L0 - (lo & ~63) > p.n_splits * p.chunk;
+  const int L = bad ? 0 : L0;
+  const int kstart = (lo & ~63) + split * p.chunk;
+  const int kend = min(L, kstart + p.chunk);
+  const int klo = max(lo, kstart);
+  const int n_tiles = kend > klo ? (kend - kstart + C::TK - 1) / C::TK : 0;
+  if (bad && threadIdx.x == 0 && split == 0 && hb == 0) atomicOr(p.status, kStatusArg);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
@@ -105,7 +145,37 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   __syncthreads();
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- append + TMA producer
+    if (p.k_new != nullptr && n_tiles > 0 && pos_b >= kstart && pos_b < kend) {
+      // the step's own token: key rotated to pos_b, stored with its value at row pos_b,
+      // ordered before this CTA's tile loads (async proxy) by the fence below
+      long long row = -1;
+      if (p.page == 0) {
+        row = static_cast<long long>(kv_bh) * p.S_cache + pos_b;
+      } else {
+        const int blk = p.block_table[static_cast<long long>(b) * p.max_blocks + pos_b / p.page];
+        if (blk >= 0 && blk < p.num_blocks)
+          row = (static_cast<long long>(blk) * p.Hkv + g) * p.page + pos_b % p.page;
+        else if (lane == 0)
+          atomicOr(p.status, kStatusArg);
+      }
+      if (row >= 0) {
+        const double log2_base = log2(static_cast<double>(p.rope_base));
+        const uint4* kn = reinterpret_cast<const uint4*>(p.k_new + static_cast<long long>(kv_bh) * D);
+        const uint4* vn = reinterpret_cast<const uint4*>(p.v_new + static_cast<long long>(kv_bh) * D);
+        uint4* kd = reinterpret_cast<uint4*>(p.k_cache + row * D);
+        uint4* vd = reinterpret_cast<uint4*>(p.v_cache + row * D);
+        for (int c8 = lane; c8 < D / 8; c8 += 32) {
+          float2 cs[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) rope_cos_sin(pos_b, c8 * 4 + t, D, log2_base, cs[t].x, cs[t].y);
+          kd[c8] = rotate8(kn[c8], cs);
+          vd[c8] = vn[c8];
+        }
+        fence_proxy_async_global();
+      }
+      __syncwarp();
+    }
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -118,10 +188,27 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         mbar_expect_tx(full(st), C::STAGE);
         const int key0 = kstart + t * C::TK;
         const uint32_t dst = sKV + st * C::STAGE;
+        if (p.page == 0) {
 #pragma unroll
-        for (int db = 0; db < C::NDB; ++db) {
-          tma_load_3d(dst + db * C::BOX, &tm_k, db * 64, key0, kv_bh, full(st));
-          tma_load_3d(dst + C::TILE + db * C::BOX, &tm_v, db * 64, key0, kv_bh, full(st));
+          for (int db = 0; db < C::NDB; ++db) {
+            tma_load_3d(dst + db * C::BOX, &tm_k, db * 64, key0, kv_bh, full(st));
+            tma_load_3d(dst + C::TILE + db * C::BOX, &tm_v, db * 64, key0, kv_bh, full(st));
+          }
+        } else {
+          // one box per page; a page wholly outside [lo, L) loads the page of row pos_b in
+          // its place (its rows are masked and its V rows zeroed by the consumers)
+          for (int r0 = key0; r0 < key0 + C::TK; r0 += p.page) {
+            const int rr = (r0 + p.page <= lo || r0 >= L) ? pos_b : r0;
+            int blk = p.block_table[static_cast<long long>(b) * p.max_blocks + rr / p.page];
+            if (blk < 0 || blk >= p.num_blocks) blk = p.num_blocks;  // past the map: zeros
+            const int z = blk * p.Hkv + g;
+            const uint32_t o = static_cast<uint32_t>((r0 - key0) * 128);
+#pragma unroll
+            for (int db = 0; db < C::NDB; ++db) {
+              tma_load_3d(dst + db * C::BOX + o, &tm_k, db * 64, 0, z, full(st));
+              tma_load_3d(dst + C::TILE + db * C::BOX + o, &tm_v, db * 64, 0, z, full(st));
+            }
+          }
         }
         issued = t + 1;
       }
@@ -150,7 +237,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         const __nv_bfloat16* qv = p.q + (static_cast<long long>(b) * p.Hq + g * p.G + gh) * D;
         const float x0 = __bfloat162float(qv[2 * i]), x1 = __bfloat162float(qv[2 * i + 1]);
         float cs, sn;
-        rope_cos_sin(p.pos, i, D, log2_base, cs, sn);
+        rope_cos_sin(pos_b, i, D, log2_base, cs, sn);
         y0 = x0 * cs - x1 * sn;
         y1 = x0 * sn + x1 * cs;
       }
@@ -182,6 +269,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
       break;
     }
     const uint32_t kS = sKV + st * C::STAGE, vS = kS + C::TILE;
+    const int tile0 = kstart + t * C::TK;
+    const bool edge = tile0 < klo || tile0 + C::TK > kend;
+    if (edge) {
+      // zero the V rows of this warp's keys outside [klo, kend): P is 0 there, but 0 * NaN
+      // is not
+      for (int idx = lane; idx < 16 * (D / 8); idx += 32) {
+        const int i = idx / (D / 8), c8 = idx % (D / 8);
+        const int kk = tile0 + krow + i;
+        if (kk < klo || kk >= kend) st_shared_zero16(vS + dec_swz(krow + i, 8 * c8));
+      }
+      __syncwarp();
+    }
 
     // S^T = K . q^T over this warp's 16 keys
     float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -192,10 +291,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
       mma_bf16_16816(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
     }
     // sc[0]/[1]: key krow+r, heads 2c/2c+1; sc[2]/[3]: key krow+r+8
-    const int kg = kstart + t * C::TK + krow + r;
+    const int kg = tile0 + krow + r;
     float x0 = sc[0] * sl2, x1 = sc[1] * sl2, x2 = sc[2] * sl2, x3 = sc[3] * sl2;
-    if (kg >= kend) x0 = x1 = -INFINITY;
-    if (kg + 8 >= kend) x2 = x3 = -INFINITY;
+    if (kg >= kend || kg < klo) x0 = x1 = -INFINITY;
+    if (kg + 8 >= kend || kg + 8 < klo) x2 = x3 = -INFINITY;
     float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -228,6 +327,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
       ldsm_x4_t(vS + dec_swz(krow + (mi >> 1) * 8 + rr, 16 * mt + (mi & 1) * 8), a0, a1, a2, a3);
       mma_bf16_16816(acc[mt], a0, a1, a2, a3, b0, b1);
     }
+    if (edge) fence_proxy_async_smem();  // the generic zeroing before the next TMA fill
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(st));
   }

@@ -9,7 +9,7 @@
 namespace ra {
 
 // Sticky device-side status codes (mirrors ra_status in ropeattn.h).
-enum : unsigned int { kStatusOk = 0u, kStatusTimeout = 4u, kStatusLayout = 8u };
+enum : unsigned int { kStatusOk = 0u, kStatusTimeout = 4u, kStatusLayout = 8u, kStatusArg = 16u };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -95,6 +95,13 @@ __device__ __forceinline__ void regs_inc() {
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// orders this thread's generic-proxy global stores before later async-proxy (TMA) reads
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA

@@ -89,4 +89,33 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* __restric
   }
 }
 
+// Prefill into a KV cache: the chunk's keys k [BH, S, D] are rotated (angles from table row
+// tab_off + s, i.e. position pos0 + s) into rows pos0 + s of each [S_cache, D] slice of kc,
+// and the values v are copied to the same rows of vc. One pass over the chunk.
+__global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restrict__ k,
+                                                          const uint4* __restrict__ v,
+                                                          uint4* __restrict__ kc,
+                                                          uint4* __restrict__ vc,
+                                                          const float2* __restrict__ tab,
+                                                          long long bh_count, int S, int S_cache,
+                                                          int pos0, int D, int tab_off) {
+  const int cpr = D / 8;
+  const long long n = bh_count * S * cpr;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long row = e / cpr;
+    const int chunk = static_cast<int>(e - row * cpr);
+    const long long bh = row / S;
+    const int s = static_cast<int>(row - bh * S);
+    const long long dst = (bh * S_cache + pos0 + s) * cpr + chunk;
+    const float4* t4 =
+        reinterpret_cast<const float4*>(tab + static_cast<long long>(tab_off + s) * (D / 2) + chunk * 4);
+    const float4 a = __ldg(t4), b = __ldg(t4 + 1);
+    const float2 cs[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y),
+                          make_float2(b.z, b.w)};
+    kc[dst] = rotate8(__ldg(k + e), cs);
+    vc[dst] = __ldg(v + e);
+  }
+}
+
 }  // namespace ra

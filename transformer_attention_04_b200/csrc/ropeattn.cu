@@ -140,19 +140,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over a contiguous [BH, S, D] bf16 tensor: dims (D, S, BH), box (64, box_rows, 1),
-// 128-byte swizzle; rows past S read as zero.
-ra_status make_map(CUtensorMap* m, const void* ptr, int D, int S, long long BH, int box_rows) {
+// 3-D map over [BH, rows_alloc, D] bf16 (rows_alloc = 0: S): dims (D, S, BH), row stride D,
+// slice stride rows_alloc * D elements; box (64, box_rows, 1), 128-byte swizzle; rows past S
+// (and slices past BH) read as zero.
+ra_status make_map(CUtensorMap* m, const void* ptr, int D, int S, long long BH, int box_rows,
+                   long long rows_alloc = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
                   "cuTensorMapEncodeTiled entry point not found");
     return RA_ERR_CUDA;
   }
+  if (rows_alloc <= 0) rows_alloc = S;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
                               static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                                 static_cast<cuuint64_t>(S) * D * 2};
+                                 static_cast<cuuint64_t>(rows_alloc) * D * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
@@ -235,6 +238,312 @@ size_t decode_partials_bytes(int B, int Hq, int D, int splits) {
 
 }  // namespace
 
+
+namespace {
+
+// ------------------------------------------------------------------ prefill
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  void* k_cache;  // null: plain prefill over k, v
+  void* v_cache;
+  int S_cache;
+  int B, Hq, Hkv, Sq, Sk, D;
+  float rope_base;
+  int pos_offset;
+  int causal;
+  int window;
+};
+
+ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
+  const int B = a.B, Hq = a.Hq, Hkv = a.Hkv, Sq = a.Sq, Sk = a.Sk, D = a.D;
+  if (!a.q || !a.k || !a.v || !a.out) return RA_ERR_INVALID_ARG;
+  if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out))
+    return RA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || D < 1) return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
+  if (!(a.rope_base > 0.f) || !std::isfinite(a.rope_base) || a.pos_offset < 0)
+    return RA_ERR_INVALID_ARG;
+  if (a.window < 0 || (a.window > 0 && !a.causal)) return RA_ERR_INVALID_ARG;
+  const bool cached = a.k_cache != nullptr || a.v_cache != nullptr;
+  if (cached && (!a.k_cache || !a.v_cache || !aligned16(a.k_cache) || !aligned16(a.v_cache)))
+    return RA_ERR_INVALID_ARG;
+  const long long T = cached ? static_cast<long long>(a.pos_offset) + Sk : Sk;  // key rows attended
+  if (cached && (a.S_cache < 1 || T > a.S_cache)) return RA_ERR_INVALID_ARG;
+  if (a.causal && Sq > T) return RA_ERR_INVALID_ARG;
+  if (static_cast<long long>(a.pos_offset) + std::max<long long>(Sq, Sk) > 0x7fffffffLL)
+    return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const size_t qbytes = static_cast<size_t>(B) * Hq * Sq * D * 2;
+  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
+  if (overlap(a.out, qbytes, a.q, qbytes) || overlap(a.out, qbytes, a.k, kbytes) ||
+      overlap(a.out, qbytes, a.v, kbytes))
+    return RA_ERR_INVALID_ARG;
+  if (cached) {
+    const size_t cbytes = static_cast<size_t>(B) * Hkv * a.S_cache * D * 2;
+    for (const void* c : {static_cast<const void*>(a.k_cache), static_cast<const void*>(a.v_cache)})
+      if (overlap(c, cbytes, a.q, qbytes) || overlap(c, cbytes, a.k, kbytes) ||
+          overlap(c, cbytes, a.v, kbytes) || overlap(c, cbytes, a.out, qbytes))
+        return RA_ERR_INVALID_ARG;
+    if (overlap(a.k_cache, cbytes, a.v_cache, cbytes)) return RA_ERR_INVALID_ARG;
+  }
+  const int G = Hq / Hkv;
+  const int n_slots = (G % 2 == 0) ? 2 : 1;
+  const int n_qtiles = (Sq + 127) / 128;
+  const long long n_units = static_cast<long long>(n_qtiles) * B * Hkv * (G / n_slots);
+  if (n_units > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL)
+    return RA_ERR_UNSUPPORTED;
+
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+
+  // workspace: rotated keys (plain prefill only), then the (cos, sin) table for positions
+  // pos_offset + tab_lo .. pos_offset + Sk - 1 (covers every query and new key position)
+  const int tab_lo = std::min(0, Sk - Sq);
+  const int tab_len = Sk - tab_lo;
+  const size_t krot_bytes = cached ? 0 : (kbytes + 255) & ~static_cast<size_t>(255);
+  const size_t tab_bytes = static_cast<size_t>(tab_len) * (D / 2) * sizeof(float2);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, krot_bytes + tab_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+  void* k_rot = ws;
+  float2* tab = reinterpret_cast<float2*>(static_cast<char*>(ws) + krot_bytes);
+
+  // a1: angles -> (cos, sin) table;  a2: K -> K' once (into the cache, with V, when cached)
+  ra::rope_table_kernel<<<grid_for(static_cast<long long>(tab_len) * (D / 2), 256, ds->num_sms),
+                          256, 0, s>>>(tab, static_cast<long long>(a.pos_offset) + tab_lo, tab_len,
+                                       D, a.rope_base);
+  const long long krows = static_cast<long long>(B) * Hkv * Sk;
+  if (cached)
+    ra::cache_write_kernel<<<grid_for(krows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
+        static_cast<const uint4*>(a.k), static_cast<const uint4*>(a.v),
+        static_cast<uint4*>(a.k_cache), static_cast<uint4*>(a.v_cache), tab,
+        static_cast<long long>(B) * Hkv, Sk, a.S_cache, a.pos_offset, D, -tab_lo);
+  else
+    ra::rope_rotate_kernel<true><<<grid_for(krows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
+        static_cast<const uint4*>(a.k), static_cast<uint4*>(k_rot), tab, krows, Sk, D, 0, -tab_lo,
+        a.rope_base);
+
+  CUtensorMap tq, tk, tv;
+  const long long bkv = static_cast<long long>(B) * Hkv;
+  rs = make_map(&tq, a.q, D, Sq, static_cast<long long>(B) * Hq, 128);
+  if (rs == RA_OK)
+    rs = cached ? make_map(&tk, a.k_cache, D, static_cast<int>(T), bkv, 128, a.S_cache)
+                : make_map(&tk, k_rot, D, Sk, bkv, 128);
+  if (rs == RA_OK)
+    rs = cached ? make_map(&tv, a.v_cache, D, static_cast<int>(T), bkv, 128, a.S_cache)
+                : make_map(&tv, a.v, D, Sk, bkv, 128);
+  if (rs == RA_OK) {
+    ra::FwdParams p;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.tab = tab;
+    p.status = ds->status;
+    p.wait_limit = g_wait_limit.load();
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Sk = static_cast<int>(T);
+    p.G = G;
+    p.n_slots = n_slots;
+    p.ppg = G / n_slots;
+    p.n_qtiles = n_qtiles;
+    p.causal = a.causal ? 1 : 0;
+    p.window = a.window;
+    p.q_tab_off = (Sk - Sq) - tab_lo;
+    p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+    // one CTA per work unit; blockIdx order is longest causal extent first
+    const dim3 grid(static_cast<unsigned>(n_units));
+    const int pi = prof_start(0, s);
+    if (D == 64)
+      ra::attn_fwd_sm100_kernel<64><<<grid, 384, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
+    else
+      ra::attn_fwd_sm100_kernel<128><<<grid, 384, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
+    prof_stop(0, pi, s);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) rs = cuda_fail(e, "attn_fwd launch");
+  }
+  cudaError_t ef = cudaFreeAsync(ws, s);
+  if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
+  return rs;
+}
+
+// ------------------------------------------------------------------ decode
+struct DecodeArgs {
+  const void* q = nullptr;
+  void* out = nullptr;
+  const void* k_cache = nullptr;  // contiguous [B, Hkv, S_cache, D] or pool [nb, Hkv, page, D]
+  const void* v_cache = nullptr;
+  int B = 0, Hq = 0, Hkv = 0, D = 0;
+  float rope_base = 0.f;
+  int pos = 0;                    // every sequence's position when pos_arr is null
+  const int* pos_arr = nullptr;   // device [B]
+  int max_pos = 0;
+  int window = 0;
+  int n_splits = 0;
+  int S_cache = 0;
+  int page = 0;                   // > 0: paged pool
+  const int* block_table = nullptr;
+  int max_blocks = 0, num_blocks = 0;
+  const void* k_new = nullptr;    // append (both or neither)
+  const void* v_new = nullptr;
+  bool noalloc = false;
+  const char* who = "";
+};
+
+ra_status scratch_too_small(const char* who, size_t need) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                "%s: %zu bytes of partials exceed the %zu-byte scratch", who, need,
+                kDecodeScratchBytes);
+  return RA_ERR_UNSUPPORTED;
+}
+
+ra_status decode_impl(const DecodeArgs& a, cudaStream_t s) {
+  const int B = a.B, Hq = a.Hq, Hkv = a.Hkv, D = a.D;
+  if (!a.q || !a.k_cache || !a.v_cache || !a.out) return RA_ERR_INVALID_ARG;
+  if (!aligned16(a.q) || !aligned16(a.k_cache) || !aligned16(a.v_cache) || !aligned16(a.out))
+    return RA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || a.n_splits < 0 || a.window < 0 || a.max_pos < 0)
+    return RA_ERR_INVALID_ARG;
+  if (!a.pos_arr && a.pos < 0) return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
+  if (!(a.rope_base > 0.f) || !std::isfinite(a.rope_base)) return RA_ERR_INVALID_ARG;
+  if ((a.k_new == nullptr) != (a.v_new == nullptr)) return RA_ERR_INVALID_ARG;
+  if (a.k_new && (!aligned16(a.k_new) || !aligned16(a.v_new))) return RA_ERR_INVALID_ARG;
+  const bool paged = a.page > 0;
+  long long cap = 0;
+  size_t cbytes = 0;
+  if (paged) {
+    if (64 % a.page || a.page < 8 || a.max_blocks < 1 || a.num_blocks < 1)
+      return RA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(a.block_table) & 3u) return RA_ERR_INVALID_ARG;
+    cap = static_cast<long long>(a.max_blocks) * a.page;
+    cbytes = static_cast<size_t>(a.num_blocks) * Hkv * a.page * D * 2;
+  } else {
+    if (a.S_cache < 1) return RA_ERR_INVALID_ARG;
+    cap = a.S_cache;
+    cbytes = static_cast<size_t>(B) * Hkv * a.S_cache * D * 2;
+  }
+  if (cap > 0x7fffffffLL) return RA_ERR_INVALID_ARG;
+  // per-sequence positions (and every paged or appending step) must lie inside the cache
+  if ((a.pos_arr || paged || a.k_new) && a.max_pos >= cap) return RA_ERR_INVALID_ARG;
+  if (a.max_pos > 0x7ffffffe) return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const size_t qbytes = static_cast<size_t>(B) * Hq * D * 2;
+  const size_t nbytes = static_cast<size_t>(B) * Hkv * D * 2;
+  if (overlap(a.out, qbytes, a.q, qbytes) || overlap(a.out, qbytes, a.k_cache, cbytes) ||
+      overlap(a.out, qbytes, a.v_cache, cbytes))
+    return RA_ERR_INVALID_ARG;
+  if (a.k_new) {
+    for (const void* c : {a.k_cache, a.v_cache})
+      if (overlap(c, cbytes, a.q, qbytes) || overlap(c, cbytes, a.k_new, nbytes) ||
+          overlap(c, cbytes, a.v_new, nbytes))
+        return RA_ERR_INVALID_ARG;
+    if (overlap(a.k_cache, cbytes, a.v_cache, cbytes) || overlap(a.out, qbytes, a.k_new, nbytes) ||
+        overlap(a.out, qbytes, a.v_new, nbytes))
+      return RA_ERR_INVALID_ARG;
+  }
+  const int G = Hq / Hkv;
+  const int hblocks = (G + 7) / 8;
+  if (static_cast<long long>(B) * Hkv * hblocks > 65535) return RA_ERR_UNSUPPORTED;
+  if (paged && static_cast<long long>(a.num_blocks) * Hkv > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+
+  // rows a sequence attends at most (R) and the 64-aligned span the splits must cover
+  const int L_max = static_cast<int>(std::min<long long>(cap, static_cast<long long>(a.max_pos) + 1));
+  const int R = a.window > 0 ? std::min(a.window, L_max) : L_max;
+  const int span = a.window > 0 ? R + 63 : L_max;
+  auto cut = [&](int splits, int* chunk) {
+    *chunk = ((span + splits - 1) / splits + 63) / 64 * 64;
+    return (span + *chunk - 1) / *chunk;
+  };
+  int chunk = 0;
+  if (a.noalloc && a.n_splits > 0) {
+    // an explicit split count (as clamped by the rows) must fit the scratch; checked first
+    const int req = cut(decode_splits(B, Hkv, G, span, 1, a.n_splits), &chunk);
+    if (decode_partials_bytes(B, Hq, D, req) > kDecodeScratchBytes)
+      return scratch_too_small(a.who, decode_partials_bytes(B, Hq, D, req));
+  }
+
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+  int splits = cut(decode_splits(B, Hkv, G, span, ds->num_sms, a.n_splits), &chunk);
+  void* scratch = nullptr;
+  if (a.noalloc) {
+    rs = decode_scratch(&scratch);
+    if (rs != RA_OK) return rs;
+    // automatic choice: the largest count up to the usual one whose partials fit
+    while (splits > 1 && decode_partials_bytes(B, Hq, D, splits) > kDecodeScratchBytes)
+      splits = cut(splits - 1, &chunk);
+    if (decode_partials_bytes(B, Hq, D, splits) > kDecodeScratchBytes)
+      return scratch_too_small(a.who, decode_partials_bytes(B, Hq, D, splits));
+  }
+  const size_t po_bytes =
+      (static_cast<size_t>(B) * Hq * splits * D * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  const size_t pml_bytes = static_cast<size_t>(B) * Hq * splits * sizeof(float2);
+
+  CUtensorMap tk, tv;
+  if (paged) {
+    const long long rows = static_cast<long long>(a.num_blocks) * Hkv;
+    rs = make_map(&tk, a.k_cache, D, a.page, rows, a.page);
+    if (rs == RA_OK) rs = make_map(&tv, a.v_cache, D, a.page, rows, a.page);
+  } else {
+    const long long bkv = static_cast<long long>(B) * Hkv;
+    rs = make_map(&tk, a.k_cache, D, a.S_cache, bkv, 64);
+    if (rs == RA_OK) rs = make_map(&tv, a.v_cache, D, a.S_cache, bkv, 64);
+  }
+  if (rs != RA_OK) return rs;
+
+  void* ws = scratch;
+  if (!a.noalloc) {
+    cudaError_t e = cudaMallocAsync(&ws, po_bytes + pml_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(decode partials)");
+  }
+  ra::DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.part_o = static_cast<float*>(ws);
+  p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + po_bytes);
+  p.status = ds->status;
+  p.wait_limit = g_wait_limit.load();
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = G;
+  p.cap = static_cast<int>(cap);
+  p.pos = a.pos;
+  p.pos_arr = a.pos_arr;
+  p.max_pos = a.max_pos;
+  p.window = a.window;
+  p.n_splits = splits;
+  p.chunk = chunk;
+  p.hblocks = hblocks;
+  p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+  p.rope_base = a.rope_base;
+  p.page = paged ? a.page : 0;
+  p.block_table = a.block_table;
+  p.max_blocks = a.max_blocks;
+  p.num_blocks = a.num_blocks;
+  p.k_new = static_cast<const __nv_bfloat16*>(a.k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(a.v_new);
+  p.k_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(a.k_cache));
+  p.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(a.v_cache));
+  p.S_cache = a.S_cache;
+  const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(B * Hkv * hblocks));
+  const int pi = prof_start(1, s);
+  if (D == 64)
+    ra::decode_split_kernel<64><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
+  else
+    ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
+  prof_stop(1, pi, s);
+  ra::decode_combine_kernel<<<static_cast<unsigned>(B * Hq), D, 0, s>>>(
+      p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(a.out), splits, D);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) rs = cuda_fail(e, "decode launch");
+  if (!a.noalloc) {
+    cudaError_t ef = cudaFreeAsync(ws, s);
+    if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(decode partials)");
+  }
+  return rs;
+}
+
+}  // namespace
+
 extern "C" {
 
 int rope_attn_version(void) { return 100; }
@@ -295,6 +604,12 @@ ra_status rope_attn_get_device_status(ra_stream_t stream) {
   const unsigned int zero = 0;
   if ((e = cudaMemcpy(ds->status, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(e, "clear status");
+  if (v & ra::kStatusArg) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "a per-sequence position or block-table entry was out of range; those "
+                  "sequences were not computed");
+    return RA_ERR_INVALID_ARG;
+  }
   if (v & ra::kStatusLayout) {
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
                   "kernel shared-memory base was not 1024-byte aligned; no work was done");
@@ -323,87 +638,22 @@ ra_status rope_attn_rotate(const void* x, void* x_rot, int B, int H, int S, int 
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "rope_rotate launch");
 }
 
+
 ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int Hq,
                         int Hkv, int Sq, int Sk, int D, float rope_base, int pos_offset,
                         int causal, ra_stream_t stream) {
-  if (!q || !k || !v || !out) return RA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return RA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || D < 1) return RA_ERR_INVALID_ARG;
-  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
-  if (causal && Sq > Sk) return RA_ERR_INVALID_ARG;
-  if (!(rope_base > 0.f) || !std::isfinite(rope_base) || pos_offset < 0) return RA_ERR_INVALID_ARG;
-  if (static_cast<long long>(pos_offset) + std::max(Sq, Sk) > 0x7fffffffLL) return RA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
-  const size_t qbytes = static_cast<size_t>(B) * Hq * Sq * D * 2;
-  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
-  if (overlap(out, qbytes, q, qbytes) || overlap(out, qbytes, k, kbytes) ||
-      overlap(out, qbytes, v, kbytes))
-    return RA_ERR_INVALID_ARG;
-  const int G = Hq / Hkv;
-  const int n_slots = (G % 2 == 0) ? 2 : 1;
-  const int n_qtiles = (Sq + 127) / 128;
-  const long long n_units = static_cast<long long>(n_qtiles) * B * Hkv * (G / n_slots);
-  if (n_units > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL)
-    return RA_ERR_UNSUPPORTED;
+  PrefillArgs a{q, k, v, out, nullptr, nullptr, 0, B, Hq, Hkv, Sq, Sk, D, rope_base,
+                pos_offset, causal, 0};
+  return prefill_impl(a, reinterpret_cast<cudaStream_t>(stream));
+}
 
-  DeviceState* ds = nullptr;
-  ra_status rs = device_state(&ds);
-  if (rs != RA_OK) return rs;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
-  // workspace: rotated keys, then the (cos, sin) table for positions
-  // pos_offset + tab_lo .. pos_offset + Sk - 1 (covers every query and key position)
-  const int tab_lo = std::min(0, Sk - Sq);
-  const int tab_len = Sk - tab_lo;
-  const size_t krot_bytes = (kbytes + 255) & ~static_cast<size_t>(255);
-  const size_t tab_bytes = static_cast<size_t>(tab_len) * (D / 2) * sizeof(float2);
-  void* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, krot_bytes + tab_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
-  void* k_rot = ws;
-  float2* tab = reinterpret_cast<float2*>(static_cast<char*>(ws) + krot_bytes);
-
-  // a1: angles -> (cos, sin) table;  a2: K -> K' once
-  ra::rope_table_kernel<<<grid_for(static_cast<long long>(tab_len) * (D / 2), 256, ds->num_sms),
-                          256, 0, s>>>(tab, static_cast<long long>(pos_offset) + tab_lo, tab_len,
-                                       D, rope_base);
-  const long long krows = static_cast<long long>(B) * Hkv * Sk;
-  ra::rope_rotate_kernel<true><<<grid_for(krows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
-      static_cast<const uint4*>(k), static_cast<uint4*>(k_rot), tab, krows, Sk, D, 0, -tab_lo,
-      rope_base);
-
-  CUtensorMap tq, tk, tv;
-  rs = make_map(&tq, q, D, Sq, static_cast<long long>(B) * Hq, 128);
-  if (rs == RA_OK) rs = make_map(&tk, k_rot, D, Sk, static_cast<long long>(B) * Hkv, 128);
-  if (rs == RA_OK) rs = make_map(&tv, v, D, Sk, static_cast<long long>(B) * Hkv, 128);
-  if (rs == RA_OK) {
-    ra::FwdParams p;
-    p.out = static_cast<__nv_bfloat16*>(out);
-    p.tab = tab;
-    p.status = ds->status;
-    p.wait_limit = g_wait_limit.load();
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Sk = Sk;
-    p.G = G;
-    p.n_slots = n_slots;
-    p.ppg = G / n_slots;
-    p.n_qtiles = n_qtiles;
-    p.causal = causal ? 1 : 0;
-    p.q_tab_off = (Sk - Sq) - tab_lo;
-    p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
-    // one CTA per work unit; blockIdx order is longest causal extent first
-    const dim3 grid(static_cast<unsigned>(n_units));
-    const int pi = prof_start(0, s);
-    if (D == 64)
-      ra::attn_fwd_sm100_kernel<64><<<grid, 384, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
-    else
-      ra::attn_fwd_sm100_kernel<128><<<grid, 384, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
-    prof_stop(0, pi, s);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) rs = cuda_fail(e, "attn_fwd launch");
-  }
-  cudaError_t ef = cudaFreeAsync(ws, s);
-  if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
-  return rs;
+ra_status rope_attn_prefill(const void* q, const void* k, const void* v, void* out,
+                            void* k_cache_rot, void* v_cache, int S_cache, int B, int Hq, int Hkv,
+                            int Sq, int Sk, int D, float rope_base, int pos_offset, int causal,
+                            int window, ra_stream_t stream) {
+  PrefillArgs a{q, k, v, out, k_cache_rot, v_cache, S_cache, B, Hq, Hkv, Sq, Sk, D, rope_base,
+                pos_offset, causal, window};
+  return prefill_impl(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos) {
@@ -418,72 +668,57 @@ int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos)
 ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const void* v_cache,
                            void* out, int B, int Hq, int Hkv, int Sk, int D, float rope_base,
                            int pos, int n_splits, ra_stream_t stream) {
-  if (!q || !k_cache_rot || !v_cache || !out) return RA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache_rot) || !aligned16(v_cache) || !aligned16(out))
-    return RA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Sk < 1 || D < 1 || pos < 0 || n_splits < 0)
-    return RA_ERR_INVALID_ARG;
-  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
-  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return RA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
-  const size_t qbytes = static_cast<size_t>(B) * Hq * D * 2;
-  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
-  if (overlap(out, qbytes, q, qbytes) || overlap(out, qbytes, k_cache_rot, kbytes) ||
-      overlap(out, qbytes, v_cache, kbytes))
-    return RA_ERR_INVALID_ARG;
-  const int G = Hq / Hkv;
-  const int hblocks = (G + 7) / 8;
-  if (static_cast<long long>(B) * Hkv * hblocks > 65535) return RA_ERR_UNSUPPORTED;
+  DecodeArgs a;
+  a.q = q; a.out = out; a.k_cache = k_cache_rot; a.v_cache = v_cache;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.rope_base = rope_base;
+  a.pos = pos; a.max_pos = pos; a.n_splits = n_splits; a.S_cache = Sk;
+  a.who = "rope_attn_decode";
+  return decode_impl(a, reinterpret_cast<cudaStream_t>(stream));
+}
 
-  DeviceState* ds = nullptr;
-  ra_status rs = device_state(&ds);
-  if (rs != RA_OK) return rs;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+ra_status rope_attn_decode_noalloc(const void* q, const void* k_cache_rot, const void* v_cache,
+                                   void* out, int B, int Hq, int Hkv, int Sk, int D,
+                                   float rope_base, int pos, int n_splits, ra_stream_t stream) {
+  DecodeArgs a;
+  a.q = q; a.out = out; a.k_cache = k_cache_rot; a.v_cache = v_cache;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.rope_base = rope_base;
+  a.pos = pos; a.max_pos = pos; a.n_splits = n_splits; a.S_cache = Sk;
+  a.noalloc = true;
+  a.who = "rope_attn_decode_noalloc";
+  return decode_impl(a, reinterpret_cast<cudaStream_t>(stream));
+}
 
-  const int L = std::min(Sk, pos + 1);
-  int splits = decode_splits(B, Hkv, G, L, ds->num_sms, n_splits);
-  const int chunk = ((L + splits - 1) / splits + 63) / 64 * 64;
-  splits = (L + chunk - 1) / chunk;
+ra_status rope_attn_decode_step(const void* q, const void* k_new, const void* v_new,
+                                void* k_cache_rot, void* v_cache, void* out, const int* pos,
+                                int B, int Hq, int Hkv, int S_cache, int D, float rope_base,
+                                int max_pos, int window, int n_splits, ra_stream_t stream) {
+  if (!pos) return RA_ERR_INVALID_ARG;
+  DecodeArgs a;
+  a.q = q; a.out = out; a.k_cache = k_cache_rot; a.v_cache = v_cache;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.rope_base = rope_base;
+  a.pos_arr = pos; a.max_pos = max_pos; a.window = window; a.n_splits = n_splits;
+  a.S_cache = S_cache;
+  a.k_new = k_new; a.v_new = v_new;
+  a.who = "rope_attn_decode_step";
+  return decode_impl(a, reinterpret_cast<cudaStream_t>(stream));
+}
 
-  const size_t po_bytes = static_cast<size_t>(B) * Hq * splits * D * sizeof(float);
-  const size_t pml_bytes = static_cast<size_t>(B) * Hq * splits * sizeof(float2);
-  void* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, po_bytes + pml_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(decode partials)");
-
-  CUtensorMap tk, tv;
-  rs = make_map(&tk, k_cache_rot, D, Sk, static_cast<long long>(B) * Hkv, 64);
-  if (rs == RA_OK) rs = make_map(&tv, v_cache, D, Sk, static_cast<long long>(B) * Hkv, 64);
-  if (rs == RA_OK) {
-    ra::DecParams p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.part_o = static_cast<float*>(ws);
-    p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + po_bytes);
-    p.status = ds->status;
-    p.wait_limit = g_wait_limit.load();
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.Sk = Sk;
-    p.L = L;
-    p.pos = pos;
-    p.n_splits = splits;
-    p.chunk = chunk;
-    p.hblocks = hblocks;
-    p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
-    p.rope_base = rope_base;
-    const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(B * Hkv * hblocks));
-    const int pi = prof_start(1, s);
-    if (D == 64)
-      ra::decode_split_kernel<64><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
-    else
-      ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
-    prof_stop(1, pi, s);
-    ra::decode_combine_kernel<<<static_cast<unsigned>(B * Hq), D, 0, s>>>(
-        p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(out), splits, D);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) rs = cuda_fail(e, "decode launch");
-  }
-  cudaError_t ef = cudaFreeAsync(ws, s);
-  if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(decode partials)");
-  return rs;
+ra_status rope_attn_decode_paged(const void* q, const void* k_new, const void* v_new,
+                                 void* k_pool_rot, void* v_pool, const int* block_table,
+                                 void* out, const int* pos, int B, int Hq, int Hkv, int D,
+                                 int page_size, int max_blocks_per_seq, int num_blocks,
+                                 float rope_base, int max_pos, int window, int n_splits,
+                                 ra_stream_t stream) {
+  if (!pos || !block_table || page_size < 1) return RA_ERR_INVALID_ARG;
+  DecodeArgs a;
+  a.q = q; a.out = out; a.k_cache = k_pool_rot; a.v_cache = v_pool;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.rope_base = rope_base;
+  a.pos_arr = pos; a.max_pos = max_pos; a.window = window; a.n_splits = n_splits;
+  a.page = page_size; a.block_table = block_table; a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.k_new = k_new; a.v_new = v_new;
+  a.who = "rope_attn_decode_paged";
+  return decode_impl(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 #ifdef RA_TRACE
@@ -494,87 +729,5 @@ RA_API int rope_attn_trace_read(void* host, size_t bytes) {
                                                                                       : RA_ERR_CUDA;
 }
 #endif
-
-ra_status rope_attn_decode_noalloc(const void* q, const void* k_cache_rot, const void* v_cache,
-                                   void* out, int B, int Hq, int Hkv, int Sk, int D,
-                                   float rope_base, int pos, int n_splits, ra_stream_t stream) {
-  if (!q || !k_cache_rot || !v_cache || !out) return RA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache_rot) || !aligned16(v_cache) || !aligned16(out))
-    return RA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Sk < 1 || D < 1 || pos < 0 || n_splits < 0)
-    return RA_ERR_INVALID_ARG;
-  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
-  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return RA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
-  const size_t qbytes = static_cast<size_t>(B) * Hq * D * 2;
-  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
-  if (overlap(out, qbytes, q, qbytes) || overlap(out, qbytes, k_cache_rot, kbytes) ||
-      overlap(out, qbytes, v_cache, kbytes))
-    return RA_ERR_INVALID_ARG;
-  const int G = Hq / Hkv;
-  const int hblocks = (G + 7) / 8;
-  if (static_cast<long long>(B) * Hkv * hblocks > 65535) return RA_ERR_UNSUPPORTED;
-  const int L = std::min(Sk, pos + 1);
-  // an explicit split count (as clamped by L) must fit the scratch; checked before any CUDA call
-  if (n_splits > 0) {
-    const int req = std::min(n_splits, std::max(1, (L + 63) / 64));
-    if (decode_partials_bytes(B, Hq, D, req) > kDecodeScratchBytes) {
-      std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
-                    "rope_attn_decode_noalloc: %zu bytes of partials exceed the %zu-byte scratch",
-                    decode_partials_bytes(B, Hq, D, req), kDecodeScratchBytes);
-      return RA_ERR_UNSUPPORTED;
-    }
-  }
-
-  DeviceState* ds = nullptr;
-  ra_status rs = device_state(&ds);
-  if (rs != RA_OK) return rs;
-  void* scratch = nullptr;
-  rs = decode_scratch(&scratch);
-  if (rs != RA_OK) return rs;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
-  int splits = decode_splits(B, Hkv, G, L, ds->num_sms, n_splits);
-  // automatic choice: the largest count up to the usual one whose partials fit the scratch
-  while (splits > 1 && decode_partials_bytes(B, Hq, D, splits) > kDecodeScratchBytes) --splits;
-  const int chunk = ((L + splits - 1) / splits + 63) / 64 * 64;
-  splits = (L + chunk - 1) / chunk;
-  if (decode_partials_bytes(B, Hq, D, splits) > kDecodeScratchBytes) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
-                  "rope_attn_decode_noalloc: %zu bytes of partials exceed the %zu-byte scratch",
-                  decode_partials_bytes(B, Hq, D, splits), kDecodeScratchBytes);
-    return RA_ERR_UNSUPPORTED;
-  }
-  const size_t po_bytes =
-      (static_cast<size_t>(B) * Hq * splits * D * sizeof(float) + 255) & ~static_cast<size_t>(255);
-
-  CUtensorMap tk, tv;
-  rs = make_map(&tk, k_cache_rot, D, Sk, static_cast<long long>(B) * Hkv, 64);
-  if (rs == RA_OK) rs = make_map(&tv, v_cache, D, Sk, static_cast<long long>(B) * Hkv, 64);
-  if (rs != RA_OK) return rs;
-  ra::DecParams p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.part_o = static_cast<float*>(scratch);
-  p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(scratch) + po_bytes);
-  p.status = ds->status;
-  p.wait_limit = g_wait_limit.load();
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.Sk = Sk;
-  p.L = L;
-  p.pos = pos;
-  p.n_splits = splits;
-  p.chunk = chunk;
-  p.hblocks = hblocks;
-  p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
-  p.rope_base = rope_base;
-  const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(B * Hkv * hblocks));
-  if (D == 64)
-    ra::decode_split_kernel<64><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
-  else
-    ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
-  ra::decode_combine_kernel<<<static_cast<unsigned>(B * Hq), D, 0, s>>>(
-      p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(out), splits, D);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? RA_OK : cuda_fail(e, "decode (no-alloc) launch");
-}
 
 }  // extern "C"
