@@ -73,3 +73,12 @@ def test_reference_arm_rank0_only_prints():
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_window_pair_count():
+    # the FLOP count of the sliding-window measurement: pairs (i, j) with i-W < j <= i
+    sys.path.insert(0, ROOT)
+    import bench
+    for S, W in [(1, 1), (10, 3), (10, 10), (10, 0), (7, 20), (300, 64)]:
+        brute = sum(1 for i in range(S) for j in range(S) if j <= i and (W == 0 or j > i - W))
+        assert bench.window_pairs(S, W) == brute
