@@ -321,8 +321,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       auto vslot = [](int j) { return (2 * j + 1) % C::NSLOT; };
       auto vpar = [](int j) { return static_cast<uint32_t>(((2 * j + 1) / C::NSLOT) & 1); };
       const long long lim = p.wait_limit;
-      bool ok = mbar_wait(bar(C::B_QREADY + 0), 0, lim, abort_flag, p.status) &&
-                mbar_wait(bar(C::B_FULL + kslot(0)), kpar(0), lim, abort_flag, p.status);
+      bool ok = mbar_wait(bar(C::B_FULL + kslot(0)), kpar(0), lim, abort_flag, p.status);
+      ok = ok && mbar_wait(bar(C::B_QREADY + 0), 0, lim, abort_flag, p.status);
       if (ok) {
         issue_s(0, kslot(0));
         umma_commit(bar(C::B_SFULL + 0));
@@ -393,21 +393,36 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t tO = tmem + t_lane + C::col_o(s);
     const long long lim = p.wait_limit;
 
-    // a3: rotate this row of Q_s in shared memory (128-byte swizzled layout of the TMA box)
+    // a3: rotate the warp's 32 rows of Q_s in shared memory (128-byte swizzled layout of
+    // the TMA box). D/8 lanes share a row, one 16-byte chunk (4 pairs) each, so every table
+    // load of the warp reads whole consecutive table rows (coalesced); all loads of the warp
+    // are issued before the first rotation.
     bool ok = mbar_wait_warp(bar(C::B_QFULL + s), 0, lim, abort_flag, p.status);
-    if (ok && qrow < p.Sq) {
-      const float4* trow = reinterpret_cast<const float4*>(
-          p.tab + static_cast<long long>(p.q_tab_off + qrow) * (D / 2));
-      uint8_t* qrow_base = smem + C::OFF_Q + s * C::TILE + r * 128;
+    if (ok) {
+      constexpr int CPR = D / 8;        // 16-byte chunks per row
+      constexpr int RPS = 32 / CPR;     // rows per warp step
+      constexpr int NSTEP = 32 / RPS;   // steps for the warp's 32 rows
+      const int k = lane % CPR, kb = k >> 3, c = k & 7;
+      float4 t[NSTEP][2];
 #pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb) {
+      for (int st = 0; st < NSTEP; ++st) {
+        const int rr = qd * 32 + st * RPS + lane / CPR;
+        const int qr = min(q0 + rr, p.Sq - 1);  // rows past Sq read a valid row, unused
+        const float4* trow = reinterpret_cast<const float4*>(
+            p.tab + static_cast<long long>(p.q_tab_off + qr) * (D / 2));
+        t[st][0] = __ldg(trow + 2 * k);
+        t[st][1] = __ldg(trow + 2 * k + 1);
+      }
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4* ptr = reinterpret_cast<uint4*>(qrow_base + kb * C::BLK + ((c ^ (r & 7)) << 4));
-          const int pair0 = kb * 32 + c * 4;
-          const float4 a = __ldg(trow + pair0 / 2), bq = __ldg(trow + pair0 / 2 + 1);
-          const float2 cs[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w),
-                                make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
+      for (int st = 0; st < NSTEP; ++st) {
+        const int rr = qd * 32 + st * RPS + lane / CPR;
+        if (q0 + rr < p.Sq) {
+          uint4* ptr = reinterpret_cast<uint4*>(smem + C::OFF_Q + s * C::TILE + kb * C::BLK +
+                                                rr * 128 + ((c ^ (rr & 7)) << 4));
+          const float2 cs[4] = {make_float2(t[st][0].x, t[st][0].y),
+                                make_float2(t[st][0].z, t[st][0].w),
+                                make_float2(t[st][1].x, t[st][1].y),
+                                make_float2(t[st][1].z, t[st][1].w)};
           *ptr = rotate8(*ptr, cs);
         }
       }
