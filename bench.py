@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--prewarm-s", type=float, default=0.5,
+                    help="seconds of untimed steps before the counted warm-up (0 for profiler runs)")
     ap.add_argument("--skip-next", action="store_true",
                     help="skip the sliding-window / KV-cache / paged decode measurements")
     ap.add_argument("--profile-leg", choices=["prefill", "decode"], default=None,
@@ -327,8 +329,9 @@ def run_ours(args):
     vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
     sampler = ClockSampler(vis[local] if local < len(vis) else local).start()
     # a freshly leased GPU runs its first ~50 ms of work slow (clock and power ramp): steps
-    # are run untimed for at least PREWARM_S seconds before the counted warm-up steps
-    prewarm(step, PREWARM_S)
+    # are run untimed for at least --prewarm-s seconds before the counted warm-up steps
+    if args.prewarm_s > 0:
+        prewarm(step, args.prewarm_s)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -423,9 +426,6 @@ def window_pairs(S: int, W: int) -> int:
     if W <= 0 or W >= S:
         return S * (S + 1) // 2
     return W * (W + 1) // 2 + (S - W) * W
-
-
-PREWARM_S = 0.5
 
 
 def prewarm(fn, seconds: float) -> int:
