@@ -298,3 +298,41 @@ def test_paged_bad_block_is_reported():
     assert not torch.equal(gpk[blk0, :, 100 % page].cpu(), pk[blk0, :, 100 % page])
     changed = (gpk.cpu().view(torch.int16) != pk.view(torch.int16)).any(dim=(1, 2, 3))
     assert int(changed.sum()) == 1
+
+
+# ----------------------------------------------------------------- head dimension 64
+
+@pytest.mark.parametrize("W", [0, 50])
+def test_decode_step_and_paged_d64(W):
+    B, Hq, Hkv, cap, D, page = 3, 12, 3, 512, 64, 32
+    pos = [511, 200, 31]
+    q, kn, vn, kc, vc = _decode_case(90, B, Hq, Hkv, cap, D, pos)
+    pk, pv, table = _to_pool(kc, vc, page, 3, 91)
+    gpos = torch.tensor(pos, dtype=torch.int32, device="cuda")
+    a = ra.rope_attn_decode_step(q.cuda(), kc.cuda(), vc.cuda(), gpos, max(pos), 10000.0,
+                                 kn.cuda(), vn.cuda(), window=W)
+    b = ra.rope_attn_decode_paged(q.cuda(), pk.cuda(), pv.cuda(), table.cuda(), gpos, max(pos),
+                                  10000.0, kn.cuda(), vn.cuda(), window=W)
+    _ok()
+    assert torch.equal(a, b)
+    want, _, _ = oracle.rope_attn_decode_step(to_f64(q), to_f64(kn), to_f64(vn), to_f64(kc),
+                                              to_f64(vc), 10000.0, pos, W)
+    assert_parity(a, want, f"d64 W={W}")
+
+
+def test_chunked_prefill_d64_non_multiple_of_tile():
+    B, Hq, Hkv, D, cap, P, Sk = 1, 6, 2, 64, 700, 250, 333
+    ctx_k, ctx_v = _bf16((B, Hkv, P, D), 92), _bf16((B, Hkv, P, D), 93)
+    q, k, v = _bf16((B, Hq, Sk, D), 94), _bf16((B, Hkv, Sk, D), 95), _bf16((B, Hkv, Sk, D), 96)
+    kc_in = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16)
+    vc_in = torch.zeros_like(kc_in)
+    kc_in[:, :, :P] = torch.from_numpy(oracle.rope_rotate(to_f64(ctx_k), np.arange(P),
+                                                          10000.0)).to(torch.bfloat16)
+    vc_in[:, :, :P] = ctx_v
+    kc, vc = kc_in.cuda(), vc_in.cuda()
+    out = ra.rope_attn_prefill(q.cuda(), k.cuda(), v.cuda(), 10000.0, P, True, window=100,
+                               k_cache_rot=kc, v_cache=vc)
+    _ok()
+    want, _, _ = oracle.rope_attn_prefill_cached(to_f64(q), to_f64(k), to_f64(v), to_f64(kc_in),
+                                                 to_f64(vc_in), 10000.0, P, window=100)
+    assert_parity(out, want, "chunked d64 window")
