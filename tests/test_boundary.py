@@ -131,3 +131,90 @@ def test_auto_splits_without_gpu(lib):
     s = lib.rope_attn_decode_auto_splits(32, 64, 8, 8192, 128, 8191)
     assert 1 <= s <= 128
     assert lib.rope_attn_decode_auto_splits(1, 1, 1, 10, 128, 9) == 1
+
+
+def test_header_is_plain_c_and_links(tmp_path, lib):
+    # include/ropeattn.h compiles as C99 with warnings as errors, and a C caller links
+    # against the library (no C++ or CUDA types cross the boundary)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(
+        '#include "ropeattn.h"\n'
+        "#include <stdio.h>\n"
+        "int main(void) {\n"
+        "  ra_status s = rope_attn_fwd(0, 0, 0, 0, 1, 1, 1, 1, 1, 64, 10000.f, 0, 1, 0);\n"
+        "  printf(\"%d %d %s\\n\", (int)s, rope_attn_version(), rope_attn_status_string(s));\n"
+        "  return s == RA_ERR_INVALID_ARG ? 0 : 1;\n"
+        "}\n")
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(ra.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir,
+                        "-lropeattn", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert run.stdout.split()[1] == "100"
+
+
+def prefill(lib, q=FAKE, k=FAKE + (1 << 40), v=FAKE + (2 << 40), out=FAKE + (3 << 40),
+            kc=0, vc=0, S_cache=0, B=1, Hq=4, Hkv=2, Sq=16, Sk=16, D=64, base=10000.0, pos=0,
+            causal=1, window=0):
+    return lib.rope_attn_prefill(q, k, v, out, kc, vc, S_cache, B, Hq, Hkv, Sq, Sk, D, base, pos,
+                                 causal, window, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(window=-1),                                           # negative window
+    dict(window=8, causal=0),                                  # a window needs the causal mask
+    dict(kc=FAKE + (4 << 40)),                                 # one cache without the other
+    dict(kc=FAKE + (4 << 40), vc=FAKE + (5 << 40), S_cache=0),  # caches without a row count
+    dict(kc=FAKE + (4 << 40), vc=FAKE + (5 << 40), S_cache=20, pos=8),  # pos_offset + Sk > S_cache
+    dict(kc=FAKE + (4 << 40) + 8, vc=FAKE + (5 << 40), S_cache=64),     # misaligned cache
+    dict(kc=FAKE + (3 << 40), vc=FAKE + (5 << 40), S_cache=64),         # cache overlaps out
+])
+def test_prefill_rejects(lib, kw):
+    assert prefill(lib, **kw) == ra.RA_ERR_INVALID_ARG
+
+
+def step(lib, q=FAKE, kn=0, vn=0, kc=FAKE + (1 << 40), vc=FAKE + (2 << 40), out=FAKE + (3 << 40),
+         pos=FAKE + (4 << 40), B=2, Hq=4, Hkv=2, S_cache=128, D=64, base=10000.0, max_pos=100,
+         window=0, splits=0):
+    return lib.rope_attn_decode_step(q, kn, vn, kc, vc, out, pos, B, Hq, Hkv, S_cache, D, base,
+                                     max_pos, window, splits, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(pos=0),                           # positions are required
+    dict(max_pos=128),                     # positions must lie inside the cache
+    dict(max_pos=-1),
+    dict(kn=FAKE + (5 << 40)),             # new key without new value
+    dict(window=-2),
+    dict(splits=-1),
+    dict(Hq=3),                            # Hq % Hkv != 0
+])
+def test_decode_step_rejects(lib, kw):
+    assert step(lib, **kw) == ra.RA_ERR_INVALID_ARG
+
+
+def paged(lib, q=FAKE, kp=FAKE + (1 << 40), vp=FAKE + (2 << 40), table=FAKE + (3 << 40),
+          out=FAKE + (4 << 40), pos=FAKE + (5 << 40), B=2, Hq=4, Hkv=2, D=64, page=16, maxb=8,
+          nb=16, base=10000.0, max_pos=100, window=0, splits=0):
+    return lib.rope_attn_decode_paged(q, 0, 0, kp, vp, table, out, pos, B, Hq, Hkv, D, page, maxb,
+                                      nb, base, max_pos, window, splits, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(page=12),                         # pages must divide 64 ...
+    dict(page=4),                          # ... and hold at least 8 rows
+    dict(table=0),
+    dict(max_pos=128),                     # 8 blocks x 16 rows hold positions 0..127
+    dict(nb=0),
+    dict(maxb=0),
+])
+def test_decode_paged_rejects(lib, kw):
+    assert paged(lib, **kw) == ra.RA_ERR_INVALID_ARG
