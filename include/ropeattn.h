@@ -73,7 +73,7 @@ RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void
  * Prefill with a sliding window and/or straight into a KV cache (chunked prefill).
  *
  * window W > 0 (causal only): key j is visible to query row i iff
- *   p_q(i) - W < p_k(j) <= p_q(i), i.e. each token sees its nearest W tokens, itself included
+ *   p_q(i) - W < p_k(j) <= p_q(i), i.e. the W positions ending at the query's own
  * ("Building Self-Attention and Transformer Engines" (codingpancake.com), §6.4 "Sliding
  * Window Attention (SWA) in Mistral 7B" and FAQ Q10). W = 0: no window. KV tiles wholly
  * outside every row's window are skipped.

@@ -39,8 +39,8 @@ Readings where the pages leave a step open (each also listed in the design notes
 * Decode: the single query at absolute position ``pos`` attends cache rows
   0..min(Sk, pos+1)-1, which hold keys that were already rotated when written.
 * Sliding window ("Building Self-Attention and Transformer Engines", §6.4 "Sliding Window
-  Attention (SWA) in Mistral 7B" and FAQ Q10: each token attends only to the nearest W
-  preceding tokens): a query at position p sees the keys at positions p-W+1 .. p, itself
+  Attention (SWA) in Mistral 7B" and FAQ Q10, which limit every token to a window of W
+  positions behind it): a query at position p sees the keys at positions p-W+1 .. p, its own
   included, so W = 1 attends only to itself; W = 0 means no window.
 """
 from __future__ import annotations
