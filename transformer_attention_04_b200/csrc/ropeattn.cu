@@ -187,7 +187,9 @@ int decode_splits(int B, int Hkv, int G, int L, int num_sms, int requested) {
   const int max_splits = std::max(1, (L + 63) / 64);
   if (requested > 0) return std::min(requested, max_splits);
   const long long base = static_cast<long long>(B) * Hkv * ((G + 7) / 8);
-  const double slots = 2.0 * num_sms;  // two decode CTAs fit on one SM
+  // Two decode CTAs fit on one SM, but one per SM already saturates HBM: waves are counted
+  // in SMs (measured on the batch-32 8k decode: 4 splits 170 us, 8 splits 174 us)
+  const double slots = static_cast<double>(num_sms);
   int best = 1;
   double best_eff = -1.0;
   for (int s = 1; s <= std::min(max_splits, 32); ++s) {
