@@ -123,11 +123,16 @@ def measured_peaks():
 
 
 def kernel_source_hash(kernel: str):
-    """sha256[:16] over the source files a kernel is compiled from."""
+    """sha256[:16] over the code of the source files a kernel is compiled from (comments
+    removed and whitespace collapsed, so only a change to the code itself counts)."""
+    import re
     h = hashlib.sha256()
     for p in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -28,8 +28,8 @@
 // thread execute in order, so S_s(j+1) never overwrites P_s(j) before PV_s(j) has read it,
 // and each commit after S_s(j) also covers PV_s(j-1) (used before rescaling O_s).
 //
-// Q is rotated in shared memory by its softmax group right after the TMA load (a3); K is
-// rotated once per call by rope_rotate_kernel into a workspace (a2), since every K tile is
+// Q is rotated in shared memory by its softmax group right after the TMA load; K is
+// rotated once per call by rope_rotate_kernel into a workspace, since every K tile is
 // re-read by S/128 query tiles.
 #pragma once
 
@@ -212,7 +212,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int off = p.Sk - p.Sq;  // query row i sits at key index i + off
   int n_kv = (p.Sk + 127) / 128;
   if (p.causal) n_kv = min(n_kv, (min(p.Sq - 1, q0 + 127) + off) / 128 + 1);
-  // a6 with a sliding window: tiles wholly below the first row's window are skipped too
+  // with a sliding window, tiles wholly below the first row's window are skipped too
   const int j_lo = (p.window > 0) ? max(0, q0 + off - p.window + 1) / 128 : 0;
   const int n_it = n_kv - j_lo;  // KV tiles this CTA visits: j_lo .. n_kv - 1
   const int ns = p.n_slots;
@@ -393,7 +393,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t tO = tmem + t_lane + C::col_o(s);
     const long long lim = p.wait_limit;
 
-    // a3: rotate the warp's 32 rows of Q_s in shared memory (128-byte swizzled layout of
+    // rotate the warp's 32 rows of Q_s in shared memory (128-byte swizzled layout of
     // the TMA box). D/8 lanes share a row, one 16-byte chunk (4 pairs) each, so every table
     // load of the warp reads whole consecutive table rows (coalesced); all loads of the warp
     // are issued before the first rotation.
@@ -449,7 +449,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_ld32(tS + 96, sr + 96);
       tmem_wait_ld();
 
-      // a6: causal / sequence-end mask, only on tiles that reach past some row's limit
+      // causal / sequence-end mask, only on tiles that reach past some row's limit
       const int kbase = (j_lo + j) * 128;
       const bool need_mask = (kbase + 128 > p.Sk) || (p.causal && kbase + 127 > q0 + off) ||
                              (p.window > 0 && kbase + p.window < q0 + 128 + off);
@@ -460,7 +460,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int c = 0; c < 128; ++c)
           if (c > lim_k || c < lo_k) sr[c] = 0xff800000u;  // -inf
       }
-      // a7: online softmax with a lazily updated reference max m. Once a row has a
+      // online softmax with a lazily updated reference max m. Once a row has a
       // reference, P is computed speculatively with it while the tile max is gathered
       // on the side; only if some row's max grew by more than 8 (log2 units) does the warp
       // redo the tile exactly (rescale O, P with the new reference). Either way every row
@@ -497,7 +497,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (upd) m = m_new;
         l *= alpha;
         if (j > 0 && __any_sync(0xffffffffu, upd)) {
-          // a8: O_s *= alpha (PV_s(j-1) has completed: it was issued before S_s(j))
+          // O_s *= alpha (PV_s(j-1) has completed: it was issued before S_s(j))
 #pragma unroll
           for (int cb = 0; cb < D; cb += 32) {
             uint32_t o[32];
@@ -522,7 +522,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0 && qd == 0) RA_STAMP(9 + 2 * s, j);
     }
 
-    // a10: epilogue O / l -> bf16
+    // epilogue O / l -> bf16
     if (ok && mbar_wait_warp(bar(C::B_OFULL + s), 0, lim, abort_flag, p.status)) {
       tc_fence_after();
       const float inv = 1.0f / l;

@@ -226,7 +226,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   const int r = lane >> 2, c = lane & 3;
   __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(smem + C::OFF_Q);
 
-  // a11 (1/3): rotate the block's (up to) 8 query rows at `pos`; rows past G are zero
+  // rotate the block's (up to) 8 query rows at `pos`; rows past G are zero
   {
     const double log2_base = log2(static_cast<double>(p.rope_base));
     for (int e = ct; e < 8 * (D / 2); e += 128) {
@@ -378,7 +378,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 }
 
-// a12: out[b, h, 0, :] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
+// the merge of the splits: out[b, h, 0, :] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
 __global__ void decode_combine_kernel(const float* __restrict__ part_o,
                                       const float2* __restrict__ part_ml,
                                       __nv_bfloat16* __restrict__ out, int n_splits, int D) {

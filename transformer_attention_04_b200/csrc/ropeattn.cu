@@ -314,7 +314,7 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
   void* k_rot = ws;
   float2* tab = reinterpret_cast<float2*>(static_cast<char*>(ws) + krot_bytes);
 
-  // a1: angles -> (cos, sin) table;  a2: K -> K' once (into the cache, with V, when cached)
+  // angles -> (cos, sin) table; then K -> K' once (into the cache, with V, when cached)
   ra::rope_table_kernel<<<grid_for(static_cast<long long>(tab_len) * (D / 2), 256, ds->num_sms),
                           256, 0, s>>>(tab, static_cast<long long>(a.pos_offset) + tab_lo, tab_len,
                                        D, a.rope_base);
