@@ -64,7 +64,7 @@ def parse_args(argv=None):
                     help="seconds of untimed steps before the counted warm-up (0 for profiler runs)")
     ap.add_argument("--skip-next", action="store_true",
                     help="skip the sliding-window / KV-cache / paged decode measurements")
-    ap.add_argument("--profile-leg", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--profile-leg", choices=["prefill", "decode", "window", "paged"], default=None,
                     help="run only this leg, warm-up + steps launches, and print no JSON "
                          "(the command that ncu captures wraps; holds only that leg's buffers)")
     a = ap.parse_args(argv)
@@ -349,8 +349,10 @@ def run_ours(args):
     barrier(world)
     torch.cuda.synchronize()
     t_start.record()
+    h0 = time.perf_counter()
     for i in range(args.steps):
         step(evs[i])
+    host_ms = (time.perf_counter() - h0) * 1e3  # enqueue time; ~ device time = host-bound
     t_end.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -390,6 +392,7 @@ def run_ours(args):
                                 "kernel": "decode_split_kernel<128>",
                                 "traffic": recorded_traffic("decode_split_kernel decode")}},
         "prefill_ms_per_call": pre_ms / K,
+        "host_enqueue_ms_per_step": host_ms / K,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
                      "peak_source": f"{peak_src} burst bf16 GEMM",
@@ -460,6 +463,36 @@ def time_calls(fn, reps: int, warm: int = 3) -> float:
     return a.elapsed_time(b) / reps
 
 
+WINDOW_W = 4096  # the sliding-window row: W = 4096 over the 32k-token workload
+PAGE = 16  # the paged row: 16-token pages
+
+
+def decode_step_inputs(Dw, rank, dev):
+    """The decode-step rows' inputs: the decode workload's q and cache, a new token per
+    sequence, positions 8191 - 128 b (4223..8191) and the cache split into 16-token pages of a
+    shuffled pool (block table a seeded permutation)."""
+    q, kc, vc = (t.to(dev) for t in make_inputs(Dw, rank_seed(rank, 1)))
+    g = torch.Generator().manual_seed(rank_seed(rank, 3))
+    kn = torch.randn(Dw.B, Dw.Hkv, 1, Dw.D, generator=g).to(torch.bfloat16).to(dev)
+    vn = torch.randn(Dw.B, Dw.Hkv, 1, Dw.D, generator=g).to(torch.bfloat16).to(dev)
+    pos_h = [Dw.Sk - 1 - 128 * b for b in range(Dw.B)]
+    pos = torch.tensor(pos_h, dtype=torch.int32, device=dev)
+    per = Dw.Sk // PAGE
+    perm = torch.randperm(Dw.B * per, generator=g).to(torch.int32)
+    table = perm.view(Dw.B, per).to(dev)
+    return q, kc, vc, kn, vn, pos, pos_h, table
+
+
+def to_pages(Dw, cache, table):
+    """Scatter a contiguous [B, Hkv, Sk, D] cache into a pool [B*Sk/PAGE, Hkv, PAGE, D] by the
+    block table."""
+    per = Dw.Sk // PAGE
+    pool = torch.empty(Dw.B * per, Dw.Hkv, PAGE, Dw.D, dtype=cache.dtype, device=cache.device)
+    pool[table.view(-1).long()] = cache.view(Dw.B, Dw.Hkv, per, PAGE, Dw.D).permute(
+        0, 2, 1, 3, 4).reshape(-1, Dw.Hkv, PAGE, Dw.D)
+    return pool
+
+
 def next_rows_leg(ra, world, rank, dev, peaks):
     """The rows after the headline path, each timed on its own with CUDA events:
     sliding-window prefill (W = 4096 over the 32k-token workload), chunked prefill into a KV
@@ -467,7 +500,7 @@ def next_rows_leg(ra, world, rank, dev, peaks):
     per-sequence positions, and the same step on a paged cache (16-token pages)."""
     res = {}
     # sliding window: FLOPs count only the allowed pairs (4*D per pair: Q.K and P.V)
-    Wl, W = LONG, 4096
+    Wl, W = LONG, WINDOW_W
     q, k, v = (t.to(dev) for t in make_inputs(Wl, rank_seed(rank, 2)))
     out = torch.empty_like(q)
     ms = time_calls(lambda: ra.rope_attn_prefill(q, k, v, Wl.rope_base, 0, True, window=W,
@@ -475,7 +508,7 @@ def next_rows_leg(ra, world, rank, dev, peaks):
     flops = 4 * Wl.D * Wl.B * Wl.Hq * window_pairs(Wl.Sq, W)
     res["sliding_window_prefill"] = _rate_entry(
         f"{Wl.name} B{Wl.B} Hq{Wl.Hq} Hkv{Wl.Hkv} S{Wl.Sq} D{Wl.D} causal, window {W}", ms, flops,
-        world, "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s")
+        world, "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s", "attn_fwd_sm100_kernel window")
     del q, k, v, out
     # chunked prefill into a cache: the headline prefill with its keys/values written out
     P = PREFILL_W
@@ -491,12 +524,7 @@ def next_rows_leg(ra, world, rank, dev, peaks):
     del q, k, v, out, kc, vc
     # decode step with append at per-sequence positions, contiguous and paged
     Dw = DECODE_W
-    q, kc, vc = (t.to(dev) for t in make_inputs(Dw, rank_seed(rank, 1)))
-    g = torch.Generator().manual_seed(rank_seed(rank, 3))
-    kn = torch.randn(Dw.B, Dw.Hkv, 1, Dw.D, generator=g).to(torch.bfloat16).to(dev)
-    vn = torch.randn(Dw.B, Dw.Hkv, 1, Dw.D, generator=g).to(torch.bfloat16).to(dev)
-    pos_h = [Dw.Sk - 1 - 128 * b for b in range(Dw.B)]  # 8191 down to 4223
-    pos = torch.tensor(pos_h, dtype=torch.int32, device=dev)
+    q, kc, vc, kn, vn, pos, pos_h, table = decode_step_inputs(Dw, rank, dev)
     rows = sum(p + 1 for p in pos_h)
     nbytes = (2 * rows * Dw.Hkv * Dw.D * 2 + 2 * Dw.B * Dw.Hq * Dw.D * 2 +
               4 * Dw.B * Dw.Hkv * Dw.D * 2)  # K,V rows read; q, out; new token read + written
@@ -507,20 +535,13 @@ def next_rows_leg(ra, world, rank, dev, peaks):
             f"(4223..8191), new token appended")
     res["decode_step_varlen_append"] = _rate_entry(work, ms, nbytes, world, "hbm",
                                                    peaks["hbm_gbs"], 1e9, "GB/s")
-    page = 16
-    per = Dw.Sk // page
-    perm = torch.randperm(Dw.B * per, generator=g).to(torch.int32)
-    table = perm.view(Dw.B, per).to(dev)
-    kp = torch.empty(Dw.B * per, Dw.Hkv, page, Dw.D, dtype=torch.bfloat16, device=dev)
-    vp = torch.empty_like(kp)
-    idx = table.view(-1).long()
-    kp[idx] = kc.view(Dw.B, Dw.Hkv, per, page, Dw.D).permute(0, 2, 1, 3, 4).reshape(-1, Dw.Hkv, page, Dw.D)
-    vp[idx] = vc.view(Dw.B, Dw.Hkv, per, page, Dw.D).permute(0, 2, 1, 3, 4).reshape(-1, Dw.Hkv, page, Dw.D)
+    kp, vp = to_pages(Dw, kc, table), to_pages(Dw, vc, table)
     del kc, vc
     ms = time_calls(lambda: ra.rope_attn_decode_paged(q, kp, vp, table, pos, max(pos_h),
                                                       Dw.rope_base, kn, vn, out=od), 50)
-    res["paged_decode_append"] = _rate_entry(work + f", {page}-token pages in a shuffled pool", ms,
-                                             nbytes, world, "hbm", peaks["hbm_gbs"], 1e9, "GB/s")
+    res["paged_decode_append"] = _rate_entry(work + f", {PAGE}-token pages in a shuffled pool", ms,
+                                             nbytes, world, "hbm", peaks["hbm_gbs"], 1e9, "GB/s",
+                                             "decode_split_kernel paged")
     del q, kp, vp, od
     torch.cuda.synchronize()
     if ra.rope_attn_get_device_status() != ra.RA_OK:
@@ -536,10 +557,16 @@ def next_rows_leg(ra, world, rank, dev, peaks):
     return res
 
 
-def _rate_entry(workload, ms, work, world, bound, peak, scale, unit):
-    return {"workload": workload, "ms_per_call": ms, "work_per_call": work, "unit": unit,
-            "bound": bound, "peak": peak, "_scale": scale,
-            "note": "inputs resident in HBM; mean over back-to-back calls (CUDA events)"}
+def _rate_entry(workload, ms, work, world, bound, peak, scale, unit, traffic_key=None):
+    e = {"workload": workload, "ms_per_call": ms, "work_per_call": work, "unit": unit,
+         "bound": bound, "peak": peak, "_scale": scale,
+         "note": "inputs resident in HBM; mean over back-to-back calls (CUDA events)"}
+    if traffic_key:
+        # DRAM bytes of the call's main kernel from its committed ncu capture (null once the
+        # kernel's code has changed since)
+        e["kernel"] = traffic_key.split()[0]
+        e["traffic"] = recorded_traffic(traffic_key)
+    return e
 
 
 def e2e_leg(ra, args, world, dev, qp, kp, vp, qd, kd, vd):
@@ -586,11 +613,25 @@ def run_profile_leg(args):
         q, k, v = (t.to(dev) for t in make_inputs(W, rank_seed(0, 0)))
         out = torch.empty_like(q)
         call = lambda: ra.rope_attn_fwd(q, k, v, W.rope_base, 0, True, out=out)
-    else:
+    elif args.profile_leg == "decode":
         W = DECODE_W
         q, k, v = (t.to(dev) for t in make_inputs(W, rank_seed(0, 1)))
         out = torch.empty_like(q)
         call = lambda: ra.rope_attn_decode(q, k, v, W.rope_base, W.decode_pos, out=out)
+    elif args.profile_leg == "window":
+        W = LONG
+        q, k, v = (t.to(dev) for t in make_inputs(W, rank_seed(0, 2)))
+        out = torch.empty_like(q)
+        call = lambda: ra.rope_attn_prefill(q, k, v, W.rope_base, 0, True, window=WINDOW_W,
+                                            out=out)
+    else:
+        W = DECODE_W
+        q, kc, vc, kn, vn, pos, pos_h, table = decode_step_inputs(W, 0, dev)
+        kp, vp = to_pages(W, kc, table), to_pages(W, vc, table)
+        del kc, vc
+        out = torch.empty_like(q)
+        call = lambda: ra.rope_attn_decode_paged(q, kp, vp, table, pos, max(pos_h), W.rope_base,
+                                                 kn, vn, out=out)
     for _ in range(args.warmup + args.steps):
         call()
     torch.cuda.synchronize()
