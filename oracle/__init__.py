@@ -10,4 +10,8 @@ from .ref import (  # noqa: F401
     rope_attn_decode_step,
     gather_pages,
     rope_attn_decode_paged,
+    rope_attn_fwd_partial,
+    merge_partials,
+    ring_shards,
+    ring_attention,
 )

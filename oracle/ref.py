@@ -38,6 +38,15 @@ Readings where the pages leave a step open (each also listed in the design notes
   every one of the D dimensions is rotated.
 * Decode: the single query at absolute position ``pos`` attends cache rows
   0..min(Sk, pos+1)-1, which hold keys that were already rotated when written.
+* Ring attention ("Building Self-Attention and Transformer Engines", §6.6 "Ring Attention"):
+  the page gives each GPU a slice of Q, K and V and passes the K/V blocks around a ring while
+  each GPU attends its queries to the block it holds; it does not say how the per-block
+  results combine. The reading here: every block yields its own normalised output and the
+  natural-log sum of exp(scores) of its allowed keys (the LSE); two results over disjoint key
+  sets combine exactly by weighting each with exp(its LSE - the LSE of both), which is the
+  same regrouping of the softmax denominator that the online softmax uses. Slices are
+  contiguous position ranges; under the causal mask a block whose keys all come after the
+  slice's queries contributes nothing and is skipped.
 * Sliding window ("Building Self-Attention and Transformer Engines", §6.4 "Sliding Window
   Attention (SWA) in Mistral 7B" and FAQ Q10, which limit every token to a window of W
   positions behind it): a query at position p sees the keys at positions p-W+1 .. p, its own
@@ -58,6 +67,10 @@ __all__ = [
     "rope_attn_decode_step",
     "gather_pages",
     "rope_attn_decode_paged",
+    "rope_attn_fwd_partial",
+    "merge_partials",
+    "ring_shards",
+    "ring_attention",
 ]
 
 
@@ -282,3 +295,108 @@ def rope_attn_decode_paged(q, k_new, v_new, k_pool_rot, v_pool, block_table, rop
         vc = gather_pages(vp, block_table, b, p + 1)[None]
         out[b:b + 1] = rope_attn_decode(q[b:b + 1], kc, vc, rope_base, p, window=window)
     return out, kp, vp
+
+
+def rope_attn_fwd_partial(q, k_rot, v, rope_base: float, q_pos0: int, k_pos0: int,
+                          causal: bool = True):
+    """One block of ring attention: queries at positions q_pos0 + i (rotated here) against
+    keys already rotated at positions k_pos0 + j, with their values.
+
+    Key j is allowed to query row i iff causal is false or k_pos0 + j <= q_pos0 + i.
+    Returns (o, lse): o [B, Hq, Sq, D] the softmax-weighted values over this block's allowed
+    keys, lse [B, Hq, Sq] = ln sum_j exp(q'_i . k'_j / sqrt(D)) over the same keys. A row with
+    no allowed key has o = 0 and lse = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_rot = np.asarray(k_rot, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Sk, _ = k_rot.shape
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    qpos = q_pos0 + np.arange(Sq, dtype=np.int64)
+    kpos = k_pos0 + np.arange(Sk, dtype=np.int64)
+    q_rot = rope_rotate(q, qpos, rope_base)
+    scale = 1.0 / np.sqrt(np.float64(D))
+    o = np.zeros((B, Hq, Sq, v.shape[-1]), dtype=np.float64)
+    lse = np.full((B, Hq, Sq), -np.inf, dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // G
+            s = (q_rot[b, h] @ k_rot[b, kv].T) * scale                   # [Sq, Sk]
+            if causal:
+                s = np.where(kpos[None, :] > qpos[:, None], -np.inf, s)
+            m = np.max(s, axis=-1)                                       # [Sq]
+            live = np.isfinite(m)
+            e = np.exp(s[live] - m[live, None])
+            tot = np.sum(e, axis=-1)
+            o[b, h, live] = (e @ v[b, kv]) / tot[:, None]
+            lse[b, h, live] = m[live] + np.log(tot)
+    return o, lse
+
+
+def merge_partials(o_a, lse_a, o_b, lse_b):
+    """Combine two partial results over disjoint key sets into the result over their union.
+
+    The union's denominator is exp(lse_a) + exp(lse_b), so its LSE is
+    L = M + ln(exp(lse_a - M) + exp(lse_b - M)) with M the larger LSE, and its output is
+    exp(lse_a - L) o_a + exp(lse_b - L) o_b. Rows where both sides are empty stay empty.
+    """
+    o_a, o_b = np.asarray(o_a, np.float64), np.asarray(o_b, np.float64)
+    lse_a, lse_b = np.asarray(lse_a, np.float64), np.asarray(lse_b, np.float64)
+    M = np.maximum(lse_a, lse_b)
+    both_empty = ~np.isfinite(M)
+    Ms = np.where(both_empty, 0.0, M)
+    tot = np.exp(lse_a - Ms) + np.exp(lse_b - Ms)
+    L = np.where(both_empty, -np.inf, Ms + np.log(np.where(both_empty, 1.0, tot)))
+    Ls = np.where(both_empty, 0.0, L)
+    w_a = np.where(both_empty, 0.0, np.exp(lse_a - Ls))
+    w_b = np.where(both_empty, 0.0, np.exp(lse_b - Ls))
+    return w_a[..., None] * o_a + w_b[..., None] * o_b, L
+
+
+def ring_shards(S: int, n: int):
+    """Contiguous slices of S positions over n ranks (the first S % n slices one longer)."""
+    q, r = divmod(S, n)
+    bounds = [0]
+    for i in range(n):
+        bounds.append(bounds[-1] + q + (1 if i < r else 0))
+    return [(bounds[i], bounds[i + 1]) for i in range(n)]
+
+
+def ring_attention(q, k, v, rope_base: float, n_ranks: int, causal: bool = True):
+    """Ring attention over n_ranks contiguous slices of one sequence (q, k, v [B, H, S, D],
+    positions 0..S-1, Sq == Sk).
+
+    Rank r rotates its own keys at their positions, then visits the K/V blocks in ring
+    order: its own (step 0), then the block of rank r-1, r-2, ... as they arrive from its
+    predecessor. Each visited block gives a partial result that is merged into the running
+    one. Under the causal mask the blocks of ranks after r lie wholly in the future of every
+    query of r and are skipped. Returns (o [B, Hq, S, D], lse [B, Hq, S]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    S = q.shape[2]
+    if k.shape[2] != S:
+        raise ValueError("ring attention here splits one sequence: Sq must equal Sk")
+    shards = ring_shards(S, n_ranks)
+    k_rot = [rope_rotate(k[:, :, a:b], np.arange(a, b), rope_base) for a, b in shards]
+    outs, lses = [], []
+    for r, (qa, qb) in enumerate(shards):
+        o_acc, lse_acc = None, None
+        for t in range(n_ranks):
+            src = (r - t) % n_ranks
+            ka, kb = shards[src]
+            if causal and src > r:
+                continue
+            o_p, lse_p = rope_attn_fwd_partial(q[:, :, qa:qb], k_rot[src], v[:, :, ka:kb],
+                                               rope_base, qa, ka, causal)
+            if o_acc is None:
+                o_acc, lse_acc = o_p, lse_p
+            else:
+                o_acc, lse_acc = merge_partials(o_acc, lse_acc, o_p, lse_p)
+        outs.append(o_acc)
+        lses.append(lse_acc)
+    return np.concatenate(outs, axis=2), np.concatenate(lses, axis=2)

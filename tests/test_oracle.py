@@ -497,3 +497,201 @@ def test_paged_decode_equals_contiguous():
         np.testing.assert_array_equal(got, want)
         for b in range(B):
             np.testing.assert_array_equal(oracle.gather_pages(kp2, table, b, 12), kc2[b])
+
+
+# ----------------------------------------------------------------- ring attention (§6.6)
+
+def _rot_brute(vec, p, base):
+    D = len(vec)
+    out = [0.0] * D
+    for i in range(D // 2):
+        a = p * base ** (-2.0 * i / D)
+        c, s = math.cos(a), math.sin(a)
+        out[2 * i] = vec[2 * i] * c - vec[2 * i + 1] * s
+        out[2 * i + 1] = vec[2 * i] * s + vec[2 * i + 1] * c
+    return out
+
+
+def _partial_brute(q, k, v, base, q_pos0, k_pos0, causal):
+    """Scalar loops and math.fsum: output and natural-log LSE of one block, with keys
+    rotated here at k_pos0 + j. Rows with no allowed key give (zeros, -inf)."""
+    B, Hq, Sq, D = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv, Sk = len(k[0]), len(k[0][0])
+    o = np.zeros((B, Hq, Sq, D))
+    lse = np.full((B, Hq, Sq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            g = h * Hkv // Hq
+            for i in range(Sq):
+                qi = _rot_brute(q[b][h][i], q_pos0 + i, base)
+                sc = []
+                for j in range(Sk):
+                    if causal and k_pos0 + j > q_pos0 + i:
+                        continue
+                    kj = _rot_brute(k[b][g][j], k_pos0 + j, base)
+                    sc.append((j, math.fsum(x * y for x, y in zip(qi, kj)) / math.sqrt(D)))
+                if not sc:
+                    continue
+                mx = max(s for _, s in sc)
+                w = [(j, math.exp(s - mx)) for j, s in sc]
+                z = math.fsum(e for _, e in w)
+                lse[b, h, i] = mx + math.log(z)
+                for d in range(D):
+                    o[b, h, i, d] = math.fsum(e * v[b][g][j][d] for j, e in w) / z
+    return o, lse
+
+
+def _rot_keys_brute(k, k_pos0, base):
+    return np.array([[[_rot_brute(row, k_pos0 + j, base) for j, row in enumerate(head)]
+                      for head in batch] for batch in k.tolist()])
+
+
+@pytest.mark.parametrize("Sq,Sk,q_pos0,k_pos0,causal", [
+    (6, 6, 0, 0, True),      # the diagonal block of a ring
+    (5, 7, 9, 0, True),      # a block wholly in the past: every key allowed
+    (6, 8, 4, 2, True),      # a block straddling the diagonal
+    (4, 6, 1, 3, True),      # the first two rows have no allowed key
+    (5, 3, 2, 11, False),    # no mask
+])
+def test_partial_block_brute_force(Sq, Sk, q_pos0, k_pos0, causal):
+    rng = np.random.default_rng(81)
+    q = rng.standard_normal((1, 4, Sq, 6))
+    k = rng.standard_normal((1, 2, Sk, 6))
+    v = rng.standard_normal((1, 2, Sk, 6))
+    base = 500.0
+    want_o, want_l = _partial_brute(q.tolist(), k.tolist(), v.tolist(), base, q_pos0, k_pos0,
+                                    causal)
+    k_rot = _rot_keys_brute(k, k_pos0, base)
+    got_o, got_l = oracle.rope_attn_fwd_partial(q, k_rot, v, base, q_pos0, k_pos0, causal)
+    np.testing.assert_allclose(got_o, want_o, atol=1e-12, rtol=0)
+    np.testing.assert_array_equal(np.isfinite(got_l), np.isfinite(want_l))
+    fin = np.isfinite(want_l)
+    np.testing.assert_allclose(got_l[fin], want_l[fin], atol=1e-12, rtol=0)
+
+
+def test_partial_single_key_lse_is_the_score():
+    # one key at the query's own position: the rotation cancels, LSE = q.k / sqrt(D)
+    rng = np.random.default_rng(82)
+    q, k, v = rng.standard_normal((1, 1, 1, 8)), rng.standard_normal((1, 1, 1, 8)), \
+        rng.standard_normal((1, 1, 1, 8))
+    k_rot = ref.rope_rotate(k, np.array([5]), 10000.0)
+    o, lse = oracle.rope_attn_fwd_partial(q, k_rot, v, 10000.0, 5, 5, True)
+    np.testing.assert_allclose(lse[0, 0, 0], float(q[0, 0, 0] @ k[0, 0, 0]) / math.sqrt(8),
+                               atol=1e-13, rtol=0)
+    np.testing.assert_allclose(o[0, 0, 0], v[0, 0, 0], atol=1e-14, rtol=0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_merge_of_key_splits_equals_whole_block(causal):
+    rng = np.random.default_rng(83)
+    Sq, Sk, q_pos0 = 9, 13, 6
+    q = rng.standard_normal((2, 4, Sq, 8))
+    k_rot = ref.rope_rotate(rng.standard_normal((2, 2, Sk, 8)), np.arange(Sk), 10000.0)
+    v = rng.standard_normal((2, 2, Sk, 8))
+    whole_o, whole_l = oracle.rope_attn_fwd_partial(q, k_rot, v, 10000.0, q_pos0, 0, causal)
+    for a in (1, 5, 12):
+        o1, l1 = oracle.rope_attn_fwd_partial(q, k_rot[:, :, :a], v[:, :, :a], 10000.0, q_pos0,
+                                              0, causal)
+        o2, l2 = oracle.rope_attn_fwd_partial(q, k_rot[:, :, a:], v[:, :, a:], 10000.0, q_pos0,
+                                              a, causal)
+        for mo, ml in (oracle.merge_partials(o1, l1, o2, l2), oracle.merge_partials(o2, l2, o1, l1)):
+            np.testing.assert_allclose(mo, whole_o, atol=1e-13, rtol=0)
+            np.testing.assert_allclose(ml, whole_l, atol=1e-13, rtol=0)
+
+
+def test_merge_with_an_empty_partial_is_identity():
+    rng = np.random.default_rng(84)
+    o, lse = rng.standard_normal((1, 2, 5, 4)), rng.standard_normal((1, 2, 5))
+    empty_o, empty_l = np.zeros_like(o), np.full_like(lse, -np.inf)
+    for mo, ml in (oracle.merge_partials(o, lse, empty_o, empty_l),
+                   oracle.merge_partials(empty_o, empty_l, o, lse)):
+        np.testing.assert_allclose(mo, o, atol=1e-15, rtol=0)
+        np.testing.assert_allclose(ml, lse, atol=1e-15, rtol=0)
+    mo, ml = oracle.merge_partials(empty_o, empty_l, empty_o, empty_l)
+    assert np.all(mo == 0) and np.all(ml == -np.inf)
+
+
+def test_ring_shards_cover_the_sequence():
+    for S, n in ((64, 4), (37, 3), (5, 5), (7, 2)):
+        sh = oracle.ring_shards(S, n)
+        assert sh[0][0] == 0 and sh[-1][1] == S and len(sh) == n
+        assert all(a[1] == b[0] for a, b in zip(sh, sh[1:]))
+        assert max(b - a for a, b in sh) - min(b - a for a, b in sh) <= 1
+
+
+@pytest.mark.parametrize("S,n", [(37, 1), (37, 2), (37, 3), (64, 4), (30, 5)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_equals_full_attention(S, n, causal):
+    rng = np.random.default_rng(85)
+    q = rng.standard_normal((2, 4, S, 8))
+    k = rng.standard_normal((2, 2, S, 8))
+    v = rng.standard_normal((2, 2, S, 8))
+    o, lse = oracle.ring_attention(q, k, v, 10000.0, n, causal)
+    np.testing.assert_allclose(o, oracle.rope_attn_fwd(q, k, v, 10000.0, 0, causal),
+                               atol=1e-13, rtol=0)
+    k_rot = ref.rope_rotate(k, np.arange(S), 10000.0)
+    _, whole_l = oracle.rope_attn_fwd_partial(q, k_rot, v, 10000.0, 0, 0, causal)
+    np.testing.assert_allclose(lse, whole_l, atol=1e-13, rtol=0)
+
+
+def test_ring_diagonal_block_is_prefill_at_its_offset():
+    rng = np.random.default_rng(86)
+    a, L = 21, 11
+    q, k, v = rng.standard_normal((1, 4, L, 8)), rng.standard_normal((1, 2, L, 8)), \
+        rng.standard_normal((1, 2, L, 8))
+    k_rot = ref.rope_rotate(k, a + np.arange(L), 10000.0)
+    o, _ = oracle.rope_attn_fwd_partial(q, k_rot, v, 10000.0, a, a, True)
+    np.testing.assert_allclose(o, oracle.rope_attn_fwd(q, k, v, 10000.0, pos_offset=a),
+                               atol=1e-13, rtol=0)
+
+
+def test_planted_ring_mistakes_are_caught(monkeypatch):
+    rng = np.random.default_rng(87)
+    q, k, v = rng.standard_normal((1, 2, 24, 4)), rng.standard_normal((1, 1, 24, 4)), \
+        rng.standard_normal((1, 1, 24, 4))
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0)
+
+    def ring_pin():
+        return np.allclose(ref.ring_attention(q, k, v, 10000.0, 3)[0], full, atol=1e-12)
+
+    def lse_pin():
+        o, l = ref.rope_attn_fwd_partial(q[:, :, :3], ref.rope_rotate(k[:, :, :3], np.arange(3),
+                                                                      10000.0),
+                                         v[:, :, :3], 10000.0, 0, 0, True)
+        want_o, want_l = _partial_brute(q[:, :, :3].tolist(), k[:, :, :3].tolist(),
+                                        v[:, :, :3].tolist(), 10000.0, 0, 0, True)
+        return np.allclose(l, want_l, atol=1e-12)
+
+    assert ring_pin() and lse_pin()
+    orig_merge, orig_partial = ref.merge_partials, ref.rope_attn_fwd_partial
+
+    # weights of the two sides swapped
+    monkeypatch.setattr(ref, "merge_partials",
+                        lambda oa, la, ob, lb: (orig_merge(oa, lb, ob, la)[0],
+                                                orig_merge(oa, la, ob, lb)[1]))
+    assert not ring_pin()
+    monkeypatch.setattr(ref, "merge_partials", orig_merge)
+
+    # key positions off by one inside a block
+    monkeypatch.setattr(ref, "rope_attn_fwd_partial",
+                        lambda q_, k_, v_, b_, qp, kp, c_=True: orig_partial(q_, k_, v_, b_, qp,
+                                                                              kp + 1, c_))
+    assert not ring_pin()
+    monkeypatch.setattr(ref, "rope_attn_fwd_partial", orig_partial)
+
+    # the causal mask dropped inside blocks
+    monkeypatch.setattr(ref, "rope_attn_fwd_partial",
+                        lambda q_, k_, v_, b_, qp, kp, c_=True: orig_partial(q_, k_, v_, b_, qp,
+                                                                              kp, False))
+    assert not ring_pin()
+    monkeypatch.setattr(ref, "rope_attn_fwd_partial", orig_partial)
+
+    # the LSE without the row max (log of the shifted sum only)
+    def lse_without_max(q_, k_, v_, b_, qp, kp, c_=True):
+        o, l = orig_partial(q_, k_, v_, b_, qp, kp, c_)
+        D = q_.shape[-1]
+        qr = ref.rope_rotate(q_, qp + np.arange(q_.shape[2]), b_)
+        s = np.einsum("bhid,bhjd->bhij", qr, np.repeat(k_, q_.shape[1] // k_.shape[1], 1))
+        return o, l - np.max(s, axis=-1) / math.sqrt(D)
+    monkeypatch.setattr(ref, "rope_attn_fwd_partial", lse_without_max)
+    assert not lse_pin()
