@@ -64,7 +64,8 @@ def parse_args(argv=None):
                     help="seconds of untimed steps before the counted warm-up (0 for profiler runs)")
     ap.add_argument("--skip-next", action="store_true",
                     help="skip the sliding-window / KV-cache / paged decode measurements")
-    ap.add_argument("--profile-leg", choices=["prefill", "decode", "window", "paged"], default=None,
+    ap.add_argument("--profile-leg", choices=["prefill", "decode", "window", "paged", "ring"],
+                    default=None,
                     help="run only this leg, warm-up + steps launches, and print no JSON "
                          "(the command that ncu captures wraps; holds only that leg's buffers)")
     a = ap.parse_args(argv)
@@ -467,6 +468,31 @@ WINDOW_W = 4096  # the sliding-window row: W = 4096 over the 32k-token workload
 PAGE = 16  # the paged row: 16-token pages
 
 
+RING_RANKS = 8  # the ring row: the 32k-token workload over 8 ranks (4096 tokens each)
+
+
+def ring_local_timed(ra, Wl, q, k, v, reps: int):
+    """Time the attention phase of an 8-rank ring run rank after rank on this GPU (every
+    rank's partial-attention calls in its ring order; key rotation and slicing excluded).
+    Returns (ms per pass, per-rank ms of the last pass)."""
+    evs = {}
+
+    def hook(r, phase):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        evs[(r, phase)] = e
+
+    ra.ring_attention_local(q, k, v, Wl.rope_base, RING_RANKS, True)
+    total, per = 0.0, []
+    for _ in range(reps):
+        evs.clear()
+        ra.ring_attention_local(q, k, v, Wl.rope_base, RING_RANKS, True, on_rank=hook)
+        torch.cuda.synchronize()
+        total += evs[(0, "start")].elapsed_time(evs[(RING_RANKS - 1, "end")])
+        per = [evs[(r, "start")].elapsed_time(evs[(r, "end")]) for r in range(RING_RANKS)]
+    return total / reps, per
+
+
 def decode_step_inputs(Dw, rank, dev):
     """The decode-step rows' inputs: the decode workload's q and cache, a new token per
     sequence, positions 8191 - 128 b (4223..8191) and the cache split into 16-token pages of a
@@ -509,6 +535,20 @@ def next_rows_leg(ra, world, rank, dev, peaks):
     res["sliding_window_prefill"] = _rate_entry(
         f"{Wl.name} B{Wl.B} Hq{Wl.Hq} Hkv{Wl.Hkv} S{Wl.Sq} D{Wl.D} causal, window {W}", ms, flops,
         world, "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s", "attn_fwd_sm100_kernel window")
+    # ring attention: the same workload, causal, as an 8-rank ring whose ranks run in turn
+    # here; per-rank times give the compute of each rank in a real ring
+    ms, per_rank = ring_local_timed(ra, Wl, q, k, v, 3)
+    L = Wl.Sk // RING_RANKS
+    e = _rate_entry(
+        f"{Wl.name} B{Wl.B} Hq{Wl.Hq} Hkv{Wl.Hkv} S{Wl.Sq} D{Wl.D} causal as a {RING_RANKS}-rank "
+        f"ring ({L} tokens per rank), ranks run in turn on one GPU", ms, Wl.flops(), world,
+        "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s")
+    e["per_rank_ms"] = per_rank
+    e["critical_rank_ms"] = max(per_rank)
+    e["exchange_bytes_per_step"] = 2 * Wl.B * Wl.Hkv * L * Wl.D * 2
+    e["kernel"] = "attn_fwd_sm100_kernel"
+    e["block_traffic"] = recorded_traffic("attn_fwd_sm100_kernel ring")
+    res["ring_long_context_8_ranks"] = e
     del q, k, v, out
     # chunked prefill into a cache: the headline prefill with its keys/values written out
     P = PREFILL_W
@@ -624,6 +664,11 @@ def run_profile_leg(args):
         out = torch.empty_like(q)
         call = lambda: ra.rope_attn_prefill(q, k, v, W.rope_base, 0, True, window=WINDOW_W,
                                             out=out)
+    elif args.profile_leg == "ring":
+        # one pass = the 36 partial-attention launches of the 8-rank ring (plus 8 rotations)
+        W = LONG
+        q, k, v = (t.to(dev) for t in make_inputs(W, rank_seed(0, 2)))
+        call = lambda: ra.ring_attention_local(q, k, v, W.rope_base, RING_RANKS, True)
     else:
         W = DECODE_W
         q, kc, vc, kn, vn, pos, pos_h, table = decode_step_inputs(W, 0, dev)

@@ -70,6 +70,40 @@ RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void
                         int causal, ra_stream_t stream);
 
 /*
+ * One block of ring attention: a slice of queries against one block of keys and values,
+ * with the result merged into a running accumulator ("Building Self-Attention and
+ * Transformer Engines" (codingpancake.com), §6.6 "Ring Attention": each GPU holds a slice of
+ * Q, K and V and attends its queries to the K/V blocks passed around the ring). The page
+ * leaves the combination of the blocks open; this call takes the exact one. Each block gives
+ * O_blk = softmax-weighted V over its allowed keys and LSE_blk = ln sum_j exp(s_ij), with
+ * s_ij = <R(q_pos0+i) q_i, k_rot_j> / sqrt(D). Two blocks over disjoint keys then combine
+ * as LSE = ln(e^LSE_a + e^LSE_b) and O = e^(LSE_a-LSE) O_a + e^(LSE_b-LSE) O_b.
+ *
+ *   q      [B, Hq,  Sq, D] bf16 (read), NOT rotated: row i is rotated to q_pos0 + i here.
+ *   k_rot  [B, Hkv, Sk, D] bf16 (read), keys already rotated to k_pos0 + j (for example by
+ *          rope_attn_rotate with pos_offset = k_pos0).   v [B, Hkv, Sk, D] bf16 (read).
+ *   o_acc  [B, Hq, Sq, D] fp32 and lse_acc [B, Hq, Sq] fp32 (natural log): the running
+ *          result, normalised (O, not O times the sum). accumulate == 0: overwritten with
+ *          this block's result. accumulate != 0: merged with their contents; an lse_acc
+ *          entry of -inf marks an empty accumulator row.
+ *   out    [B, Hq, Sq, D] bf16 or NULL: when given, also receives the merged result
+ *          (pass it on the last block).
+ *   causal: key j is allowed to query row i iff k_pos0 + j <= q_pos0 + i; requires
+ *   q_pos0 >= k_pos0, so that every row sees at least the block's first key. zero: all keys.
+ *   q_pos0, k_pos0 >= 0; q_pos0 + Sq and k_pos0 + Sk at most 2^30.
+ * o_acc, lse_acc and out must not overlap the inputs or each other; o_acc is 16-byte
+ * aligned, lse_acc 4-byte aligned. D in {64, 128}, Hq % Hkv == 0, sizes >= 1. Runs the
+ * prefill kernel of rope_attn_fwd with its fp32 epilogue (one launch, plus the RoPE table of
+ * the Sq query positions). Returns RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED or
+ * RA_ERR_CUDA.
+ */
+RA_API ra_status rope_attn_fwd_partial(const void* q, const void* k_rot, const void* v,
+                                       float* o_acc, float* lse_acc, void* out, int B, int Hq,
+                                       int Hkv, int Sq, int Sk, int D, float rope_base,
+                                       int q_pos0, int k_pos0, int causal, int accumulate,
+                                       ra_stream_t stream);
+
+/*
  * Prefill with a sliding window and/or straight into a KV cache (chunked prefill).
  *
  * window W > 0 (causal only): key j is visible to query row i iff

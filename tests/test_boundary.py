@@ -218,3 +218,34 @@ def paged(lib, q=FAKE, kp=FAKE + (1 << 40), vp=FAKE + (2 << 40), table=FAKE + (3
 ])
 def test_decode_paged_rejects(lib, kw):
     assert paged(lib, **kw) == ra.RA_ERR_INVALID_ARG
+
+
+def partial(lib, q=FAKE, k=FAKE + (1 << 40), v=FAKE + (2 << 40), o=FAKE + (3 << 40),
+            lse=FAKE + (4 << 40), out=0, B=1, Hq=4, Hkv=2, Sq=16, Sk=16, D=64, base=10000.0,
+            qp=32, kp=16, causal=1, acc=0):
+    return lib.rope_attn_fwd_partial(q, k, v, o, lse, out, B, Hq, Hkv, Sq, Sk, D, base, qp, kp,
+                                     causal, acc, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(o=0), ra.RA_ERR_INVALID_ARG),                 # the accumulator is required
+    (dict(lse=0), ra.RA_ERR_INVALID_ARG),
+    (dict(o=FAKE + (3 << 40) + 4), ra.RA_ERR_INVALID_ARG),  # o_acc not 16-byte aligned
+    (dict(lse=FAKE + (4 << 40) + 2), ra.RA_ERR_INVALID_ARG),  # lse_acc not 4-byte aligned
+    (dict(qp=15, kp=16), ra.RA_ERR_INVALID_ARG),        # causal rows before the block's first key
+    (dict(qp=-1), ra.RA_ERR_INVALID_ARG),
+    (dict(qp=2**30, kp=0), ra.RA_ERR_INVALID_ARG),      # positions past 2^30
+    (dict(Hq=3), ra.RA_ERR_INVALID_ARG),
+    (dict(o=FAKE), ra.RA_ERR_INVALID_ARG),              # o_acc overlaps q
+    (dict(lse=FAKE + (3 << 40)), ra.RA_ERR_INVALID_ARG),  # lse_acc overlaps o_acc
+    (dict(out=FAKE + (2 << 40)), ra.RA_ERR_INVALID_ARG),  # out overlaps v
+    (dict(D=96), ra.RA_ERR_UNSUPPORTED),
+])
+def test_partial_rejects(lib, kw, want):
+    assert partial(lib, **kw) == want
+
+
+def test_partial_noncausal_any_offsets_until_device(lib):
+    # without the mask a block may sit anywhere; with no GPU the call fails at the device step
+    st = partial(lib, qp=0, kp=500, causal=0)
+    assert st != ra.RA_ERR_INVALID_ARG

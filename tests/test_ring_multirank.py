@@ -1,0 +1,122 @@
+"""The ring-attention driver across real processes on CPU (gloo, world sizes 2 and 3).
+
+The driver's schedule and its point-to-point exchanges run as in a multi-GPU job; the two
+library calls it makes (key rotation, one block of attention merged into the running result)
+are replaced by fp64 stand-ins built from the oracle, so that the test checks the ring logic
+itself: which block each rank holds at each step, which blocks it skips, the positions it
+passes, the merge order and the final output. The result must equal the oracle's full
+attention over the whole sequence.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _inputs(B, Hq, Hkv, S, D, seed):
+    g = np.random.default_rng(seed)
+    return (g.standard_normal((B, Hq, S, D)), g.standard_normal((B, Hkv, S, D)),
+            g.standard_normal((B, Hkv, S, D)))
+
+
+def _worker(rank, world, port, causal, q_out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    import oracle
+    from transformer_attention_04_b200.ring import ring_attention
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    calls = []
+
+    def cpu_rotate(x, rope_base, pos_offset, out=None):
+        r = oracle.rope_rotate(x.numpy(), pos_offset + np.arange(x.shape[2]), rope_base)
+        out.copy_(torch.from_numpy(r))
+        return out
+
+    def cpu_partial(q, k_rot, v, o_acc, lse_acc, rope_base, q_pos0, k_pos0, causal=True,
+                    accumulate=False, out=None):
+        calls.append((q_pos0, k_pos0, bool(accumulate), out is not None))
+        o, lse = oracle.rope_attn_fwd_partial(q.numpy(), k_rot.numpy(), v.numpy(), rope_base,
+                                              q_pos0, k_pos0, causal)
+        if accumulate:
+            o, lse = oracle.merge_partials(o_acc.double().numpy(), lse_acc.double().numpy(), o,
+                                           lse)
+        o_acc.copy_(torch.from_numpy(o))
+        lse_acc.copy_(torch.from_numpy(lse))
+        if out is not None:
+            out.copy_(torch.from_numpy(o))
+        return out
+
+    B, Hq, Hkv, L, D = 1, 4, 2, 6, 8
+    q, k, v = _inputs(B, Hq, Hkv, world * L, D, seed=90)
+    sl = slice(rank * L, (rank + 1) * L)
+    res = ring_attention(torch.from_numpy(q[:, :, sl].copy()), torch.from_numpy(k[:, :, sl].copy()),
+                         torch.from_numpy(v[:, :, sl].copy()), 1000.0, causal=causal,
+                         partial_fn=cpu_partial, rotate_fn=cpu_rotate)
+    dist.barrier()
+    dist.destroy_process_group()
+    q_out.put((rank, res.numpy(), calls))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_attention_gloo_equals_full(world, causal):
+    sys.path.insert(0, ROOT)
+    import oracle
+
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q_out = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, causal, q_out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted([q_out.get(timeout=180) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    L = 6
+    q, k, v = _inputs(1, 4, 2, world * L, 8, seed=90)
+    want = oracle.rope_attn_fwd(q, k, v, 1000.0, 0, causal)
+    res = np.concatenate([g[1] for g in got], axis=2)
+    np.testing.assert_allclose(res, want, atol=1e-5, rtol=0)
+    for rank, _, calls in got:
+        # own block first, then the predecessors' blocks; causal skips every later rank
+        srcs = [kp // L for _, kp, _, _ in calls]
+        expect = [(rank - t) % world for t in range(world)]
+        if causal:
+            expect = [s for s in expect if s <= rank]
+        assert srcs == expect
+        assert all(qp == rank * L for qp, _, _, _ in calls)
+        assert [acc for _, _, acc, _ in calls] == [False] + [True] * (len(calls) - 1)
+        assert [o for _, _, _, o in calls] == [False] * (len(calls) - 1) + [True]
+
+
+def test_ring_steps_schedule():
+    sys.path.insert(0, ROOT)
+    from transformer_attention_04_b200.ring import ring_steps
+    assert ring_steps(0, 1, True) == [(0, 0, True)]
+    assert ring_steps(2, 4, True) == [(0, 2, True), (1, 1, True), (2, 0, True), (3, 3, False)]
+    assert [u for _, _, u in ring_steps(0, 4, True)] == [True, False, False, False]
+    assert all(u for _, _, u in ring_steps(1, 3, False))
+    # every block visits every rank once
+    for world in (2, 3, 5):
+        for r in range(world):
+            assert sorted(s for _, s, _ in ring_steps(r, world, False)) == list(range(world))

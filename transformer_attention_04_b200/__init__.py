@@ -18,6 +18,7 @@ from ._lib import (  # noqa: F401
     rope_attn_decode_paged,
     rope_attn_decode_step,
     rope_attn_fwd,
+    rope_attn_fwd_partial,
     rope_attn_get_device_status,
     rope_attn_prefill,
     rope_attn_profile_enable,
@@ -26,3 +27,4 @@ from ._lib import (  # noqa: F401
     rope_attn_set_wait_limit,
     rope_attn_version,
 )
+from .ring import ring_attention, ring_attention_local, ring_steps  # noqa: F401,E402

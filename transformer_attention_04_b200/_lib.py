@@ -24,6 +24,8 @@ SIGNATURES = {
     "rope_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
                                _P]),
     "rope_attn_rotate": (_I, [_P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "rope_attn_fwd_partial": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
+                                   _I, _P]),
     "rope_attn_decode": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "rope_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "rope_attn_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I,
@@ -136,6 +138,36 @@ def rope_attn_prefill(q, k, v, rope_base: float, pos_offset: int = 0, causal: bo
                                  S_cache, B, Hq, Hkv, Sq, Sk, D, float(rope_base), int(pos_offset),
                                  int(bool(causal)), int(window), _stream(stream))
     _raise(st, "rope_attn_prefill")
+    return out
+
+
+def rope_attn_fwd_partial(q, k_rot, v, o_acc, lse_acc, rope_base: float, q_pos0: int,
+                          k_pos0: int, causal: bool = True, accumulate: bool = False, out=None,
+                          stream=None):
+    """One ring-attention block: q [B,Hq,Sq,D] (rotated here to q_pos0+i) against keys k_rot
+    [B,Hkv,Sk,D] already rotated to k_pos0+j, and v. The block's normalised output and
+    natural-log LSE go to o_acc [B,Hq,Sq,D] / lse_acc [B,Hq,Sq] (fp32), merged with their
+    contents when ``accumulate``; ``out`` (bf16), if given, also receives the merged result."""
+    _check(q, "q")
+    if q.dim() != 4 or k_rot.dim() != 4:
+        raise ValueError("q, k_rot, v must be 4-D [B, H, S, D]")
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k_rot.shape[1], k_rot.shape[2]
+    _check(k_rot, "k_rot", (B, Hkv, Sk, D))
+    _check(v, "v", (B, Hkv, Sk, D))
+    for t, name, shape in ((o_acc, "o_acc", (B, Hq, Sq, D)), (lse_acc, "lse_acc", (B, Hq, Sq))):
+        if (not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or
+                not t.is_contiguous() or tuple(t.shape) != shape):
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of shape {shape}")
+    o = 0
+    if out is not None:
+        _check(out, "out", q.shape)
+        o = out.data_ptr()
+    st = lib().rope_attn_fwd_partial(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(),
+                                     o_acc.data_ptr(), lse_acc.data_ptr(), o, B, Hq, Hkv, Sq, Sk,
+                                     D, float(rope_base), int(q_pos0), int(k_pos0),
+                                     int(bool(causal)), int(bool(accumulate)), _stream(stream))
+    _raise(st, "rope_attn_fwd_partial")
     return out
 
 

@@ -51,6 +51,8 @@ __device__ unsigned long long g_trace[2][16][64];
   } while (0)
 #endif
 
+constexpr float kLn2 = 0.6931471805599453f;
+
 struct FwdParams {
   __nv_bfloat16* out;   // [B, Hq, Sq, D]
   const float2* tab;    // RoPE (cos, sin) table, D/2 entries per position
@@ -62,9 +64,16 @@ struct FwdParams {
   int ppg;              // CTA units per (batch, KV group, query tile) = G / n_slots
   int n_qtiles;         // ceil(Sq / 128)
   int causal;
-  int window;           // 0 = none; else key j is allowed to query row i iff j > i + Sk - Sq - window
+  int off;              // query row i sits at key index i + off (causal: key j allowed iff j <= i + off)
+  int window;           // 0 = none; else key j is allowed to query row i iff j > i + off - window
   int q_tab_off;        // table row of query row 0
   float scale_log2;     // log2(e) / sqrt(D)
+  // partial (ring) mode when o_acc is set: O / l in fp32 [B, Hq, Sq, D] and the row's natural
+  // log-sum-exp in lse_acc [B, Hq, Sq], merged into their contents when accumulate is set;
+  // `out` (bf16) is then optional and receives the merged result
+  float* o_acc;
+  float* lse_acc;
+  int accumulate;
 };
 
 template <int D>
@@ -209,7 +218,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int h0 = g * p.G + hp * p.n_slots;
   const int kv_bh = b * p.Hkv + g;
   const int q0 = qt * 128;
-  const int off = p.Sk - p.Sq;  // query row i sits at key index i + off
+  const int off = p.off;  // query row i sits at key index i + off
   int n_kv = (p.Sk + 127) / 128;
   if (p.causal) n_kv = min(n_kv, (min(p.Sq - 1, q0 + 127) + off) / 128 + 1);
   // with a sliding window, tiles wholly below the first row's window are skipped too
@@ -522,8 +531,64 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0 && qd == 0) RA_STAMP(9 + 2 * s, j);
     }
 
-    // epilogue O / l -> bf16
-    if (ok && mbar_wait_warp(bar(C::B_OFULL + s), 0, lim, abort_flag, p.status)) {
+    // epilogue, partial mode: O / l and the LSE in fp32, merged with the running result
+    // (weights exp(lse - merged lse) on each side); every row has at least one allowed key
+    if (p.o_acc != nullptr) {
+      if (ok && mbar_wait_warp(bar(C::B_OFULL + s), 0, lim, abort_flag, p.status)) {
+        tc_fence_after();
+        const long long row = static_cast<long long>(b * p.Hq + h0 + s) * p.Sq + qrow;
+        const float lse_new = (m + log2f(l)) * kLn2;
+        float w_old = 0.f, w_new = 1.0f / l, lse_out = lse_new;
+        if (p.accumulate && qrow < p.Sq) {
+          const float lse_old = p.lse_acc[row];
+          if (lse_old != -INFINITY) {
+            const float mx = fmaxf(lse_old, lse_new);
+            const float eo = expf(lse_old - mx), en = expf(lse_new - mx);
+            const float den = eo + en;
+            w_old = eo / den;
+            w_new = en / (den * l);
+            lse_out = mx + logf(den);
+          }
+        }
+        float4* acc = reinterpret_cast<float4*>(p.o_acc + row * D);
+        __nv_bfloat16* orow = p.out ? p.out + row * D : nullptr;
+#pragma unroll
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + cb, o);
+          tmem_wait_ld();
+          if (qrow < p.Sq) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * w_new;
+            if (w_old != 0.f) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 a = acc[cb / 4 + i];
+                v[4 * i + 0] += w_old * a.x;
+                v[4 * i + 1] += w_old * a.y;
+                v[4 * i + 2] += w_old * a.z;
+                v[4 * i + 3] += w_old * a.w;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              acc[cb / 4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            if (orow) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + cb);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pack_bf16(v[8 * i + 0], v[8 * i + 1]),
+                                    pack_bf16(v[8 * i + 2], v[8 * i + 3]),
+                                    pack_bf16(v[8 * i + 4], v[8 * i + 5]),
+                                    pack_bf16(v[8 * i + 6], v[8 * i + 7]));
+            }
+          }
+        }
+        if (qrow < p.Sq) p.lse_acc[row] = lse_out;
+      }
+    } else if (ok && mbar_wait_warp(bar(C::B_OFULL + s), 0, lim, abort_flag, p.status)) {
+      // epilogue O / l -> bf16
       tc_fence_after();
       const float inv = 1.0f / l;
       const uint64_t pol_out = l2_policy_evict_first();

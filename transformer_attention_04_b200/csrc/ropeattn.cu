@@ -259,6 +259,21 @@ struct PrefillArgs {
   int window;
 };
 
+// One launch of the attention kernel: one CTA per work unit (query tile, batch, KV group,
+// query-head pair); blockIdx order is longest causal extent first.
+ra_status launch_attn(const ra::FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                      const CUtensorMap& tv, int D, long long n_units, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(n_units));
+  const int pi = prof_start(0, s);
+  if (D == 64)
+    ra::attn_fwd_sm100_kernel<64><<<grid, 384, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
+  else
+    ra::attn_fwd_sm100_kernel<128><<<grid, 384, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
+  prof_stop(0, pi, s);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "attn_fwd launch");
+}
+
 ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
   const int B = a.B, Hq = a.Hq, Hkv = a.Hkv, Sq = a.Sq, Sk = a.Sk, D = a.D;
   if (!a.q || !a.k || !a.v || !a.out) return RA_ERR_INVALID_ARG;
@@ -350,19 +365,109 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.ppg = G / n_slots;
     p.n_qtiles = n_qtiles;
     p.causal = a.causal ? 1 : 0;
+    p.off = static_cast<int>(T) - Sq;  // bottom-right alignment of the queries on the keys
     p.window = a.window;
     p.q_tab_off = (Sk - Sq) - tab_lo;
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
-    // one CTA per work unit; blockIdx order is longest causal extent first
-    const dim3 grid(static_cast<unsigned>(n_units));
-    const int pi = prof_start(0, s);
-    if (D == 64)
-      ra::attn_fwd_sm100_kernel<64><<<grid, 384, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
-    else
-      ra::attn_fwd_sm100_kernel<128><<<grid, 384, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
-    prof_stop(0, pi, s);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) rs = cuda_fail(e, "attn_fwd launch");
+    p.o_acc = nullptr;
+    p.lse_acc = nullptr;
+    p.accumulate = 0;
+    rs = launch_attn(p, tq, tk, tv, D, n_units, s);
+  }
+  cudaError_t ef = cudaFreeAsync(ws, s);
+  if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
+  return rs;
+}
+
+// ------------------------------------------------------------------ ring attention block
+struct PartialArgs {
+  const void* q;
+  const void* k_rot;
+  const void* v;
+  float* o_acc;
+  float* lse_acc;
+  void* out;  // optional bf16 copy of the merged result
+  int B, Hq, Hkv, Sq, Sk, D;
+  float rope_base;
+  int q_pos0, k_pos0;
+  int causal;
+  int accumulate;
+};
+
+ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
+  const int B = a.B, Hq = a.Hq, Hkv = a.Hkv, Sq = a.Sq, Sk = a.Sk, D = a.D;
+  if (!a.q || !a.k_rot || !a.v || !a.o_acc || !a.lse_acc) return RA_ERR_INVALID_ARG;
+  if (!aligned16(a.q) || !aligned16(a.k_rot) || !aligned16(a.v) || !aligned16(a.o_acc) ||
+      (reinterpret_cast<uintptr_t>(a.lse_acc) & 3u) || (a.out && !aligned16(a.out)))
+    return RA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || D < 1) return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return RA_ERR_INVALID_ARG;
+  if (!(a.rope_base > 0.f) || !std::isfinite(a.rope_base)) return RA_ERR_INVALID_ARG;
+  // positions stay below 2^30 so that every row and key index sum fits an int
+  if (a.q_pos0 < 0 || a.k_pos0 < 0 || static_cast<long long>(a.q_pos0) + Sq > (1LL << 30) ||
+      static_cast<long long>(a.k_pos0) + Sk > (1LL << 30))
+    return RA_ERR_INVALID_ARG;
+  // under the causal mask every query row must see the block's first key
+  if (a.causal && a.q_pos0 < a.k_pos0) return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const size_t qbytes = static_cast<size_t>(B) * Hq * Sq * D * 2;
+  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
+  const size_t obytes = static_cast<size_t>(B) * Hq * Sq * D * 4;
+  const size_t lbytes = static_cast<size_t>(B) * Hq * Sq * 4;
+  for (const auto& w : {std::make_pair(static_cast<const void*>(a.o_acc), obytes),
+                        std::make_pair(static_cast<const void*>(a.lse_acc), lbytes),
+                        std::make_pair(static_cast<const void*>(a.out), a.out ? qbytes : 0)})
+    if (w.second && (overlap(w.first, w.second, a.q, qbytes) ||
+                     overlap(w.first, w.second, a.k_rot, kbytes) ||
+                     overlap(w.first, w.second, a.v, kbytes)))
+      return RA_ERR_INVALID_ARG;
+  if (overlap(a.o_acc, obytes, a.lse_acc, lbytes) ||
+      (a.out && (overlap(a.out, qbytes, a.o_acc, obytes) || overlap(a.out, qbytes, a.lse_acc, lbytes))))
+    return RA_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  const int n_slots = (G % 2 == 0) ? 2 : 1;
+  const int n_qtiles = (Sq + 127) / 128;
+  const long long n_units = static_cast<long long>(n_qtiles) * B * Hkv * (G / n_slots);
+  if (n_units > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL)
+    return RA_ERR_UNSUPPORTED;
+
+  DeviceState* ds = nullptr;
+  ra_status rs = device_state(&ds);
+  if (rs != RA_OK) return rs;
+  // workspace: the (cos, sin) table of the query positions q_pos0 .. q_pos0 + Sq - 1 (the
+  // keys arrive rotated)
+  const size_t tab_bytes = static_cast<size_t>(Sq) * (D / 2) * sizeof(float2);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, tab_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+  float2* tab = static_cast<float2*>(ws);
+  ra::rope_table_kernel<<<grid_for(static_cast<long long>(Sq) * (D / 2), 256, ds->num_sms), 256,
+                          0, s>>>(tab, a.q_pos0, Sq, D, a.rope_base);
+  CUtensorMap tq, tk, tv;
+  const long long bkv = static_cast<long long>(B) * Hkv;
+  rs = make_map(&tq, a.q, D, Sq, static_cast<long long>(B) * Hq, 128);
+  if (rs == RA_OK) rs = make_map(&tk, a.k_rot, D, Sk, bkv, 128);
+  if (rs == RA_OK) rs = make_map(&tv, a.v, D, Sk, bkv, 128);
+  if (rs == RA_OK) {
+    ra::FwdParams p;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.tab = tab;
+    p.status = ds->status;
+    p.wait_limit = g_wait_limit.load();
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Sk = Sk;
+    p.G = G;
+    p.n_slots = n_slots;
+    p.ppg = G / n_slots;
+    p.n_qtiles = n_qtiles;
+    p.causal = a.causal ? 1 : 0;
+    p.off = a.q_pos0 - a.k_pos0;  // query row i at q_pos0 + i, key j at k_pos0 + j
+    p.window = 0;
+    p.q_tab_off = 0;
+    p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+    p.o_acc = a.o_acc;
+    p.lse_acc = a.lse_acc;
+    p.accumulate = a.accumulate ? 1 : 0;
+    rs = launch_attn(p, tq, tk, tv, D, n_units, s);
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
   if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
@@ -647,6 +752,15 @@ ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   PrefillArgs a{q, k, v, out, nullptr, nullptr, 0, B, Hq, Hkv, Sq, Sk, D, rope_base,
                 pos_offset, causal, 0};
   return prefill_impl(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ra_status rope_attn_fwd_partial(const void* q, const void* k_rot, const void* v, float* o_acc,
+                                float* lse_acc, void* out, int B, int Hq, int Hkv, int Sq, int Sk,
+                                int D, float rope_base, int q_pos0, int k_pos0, int causal,
+                                int accumulate, ra_stream_t stream) {
+  PartialArgs a{q, k_rot, v, o_acc, lse_acc, out, B, Hq, Hkv, Sq, Sk, D, rope_base,
+                q_pos0, k_pos0, causal, accumulate};
+  return partial_impl(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ra_status rope_attn_prefill(const void* q, const void* k, const void* v, void* out,

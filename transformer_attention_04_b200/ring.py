@@ -1,0 +1,134 @@
+"""Ring attention over the ranks of a torch.distributed process group.
+
+"Building Self-Attention and Transformer Engines" (codingpancake.com), §6.6 "Ring Attention":
+each GPU holds a slice of one sequence's queries, keys and values. It attends its queries to
+the key/value block it holds while passing that block to the next GPU of the ring, so after
+P steps every query slice has met every block. The per-block results combine exactly through
+their log-sum-exp; `rope_attn_fwd_partial` merges each block into the running result.
+
+Slices are contiguous and of equal length L: rank r holds positions r*L .. r*L + L - 1.
+Rank r attends its own block first, then the blocks of ranks r-1, r-2, ... as they arrive
+from its predecessor. Under the causal mask, the blocks of ranks after r lie wholly in the
+future of rank r's queries and are skipped. Their transfer still happens: the ring passes
+every block on.
+
+This module is host orchestration only:
+* every arithmetic step runs in the library's kernels: `rope_attn_rotate` for the local keys,
+  `rope_attn_fwd_partial` per block;
+* the transfers are torch.distributed point-to-point operations (NCCL over NVLink between
+  GPUs). Each step's send and receive start before the step's kernel and are awaited after
+  it, so they overlap with the computation.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import _lib
+
+
+def ring_steps(rank: int, world: int, causal: bool):
+    """The (step, source rank, attended) schedule of one rank: at step t it holds the block
+    of rank (rank - t) mod world; under the causal mask blocks of later ranks are skipped."""
+    out = []
+    for t in range(world):
+        src = (rank - t) % world
+        out.append((t, src, not (causal and src > rank)))
+    return out
+
+
+def ring_attention(q, k, v, rope_base: float, causal: bool = True, group=None, out=None, *,
+                   partial_fn=None, rotate_fn=None):
+    """Exact attention of this rank's query slice over the whole ring's keys and values.
+
+    q [B, Hq, L, D], k, v [B, Hkv, L, D]: this rank's slice (positions rank*L ..), keys not
+    rotated. Returns out [B, Hq, L, D] (bf16 through the library), this slice of the
+    attention over the full sequence. Every rank of the group calls it with the same shapes.
+    ``partial_fn`` / ``rotate_fn`` replace the library calls (same signatures as
+    `rope_attn_fwd_partial` / `rope_attn_rotate`); the multi-process tests on CPU use them.
+    """
+    partial_fn = partial_fn or _lib.rope_attn_fwd_partial
+    rotate_fn = rotate_fn or _lib.rope_attn_rotate
+    distributed = dist.is_available() and dist.is_initialized()
+    world = dist.get_world_size(group) if distributed else 1
+    rank = dist.get_rank(group) if distributed else 0
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, L, D]")
+    B, Hq, L, D = q.shape
+    if k.shape[0] != B or k.shape[2:] != (L, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, L, D] with q's B, L and D")
+
+    def peer(r):
+        return r if group is None else dist.get_global_rank(group, r)
+
+    # own block (keys rotated here, values as given; read only) and two receive buffers that
+    # alternate: the block arriving at step t is attended at step t + 1, while the next one
+    # arrives in the other buffer
+    own = (torch.empty_like(k), v)
+    rotate_fn(k, rope_base, rank * L, out=own[0])
+    recv = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
+    o_acc = torch.empty((B, Hq, L, D), dtype=torch.float32, device=q.device)
+    lse_acc = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    sched = ring_steps(rank, world, causal)
+    last = max(t for t, _, used in sched if used)
+    first = True
+    nxt, prv = peer((rank + 1) % world), peer((rank - 1) % world)
+    for t, src, used in sched:
+        cur = own if t == 0 else recv[(t - 1) % 2]
+        reqs = []
+        if t < world - 1:
+            dst = recv[t % 2]
+            ops = [dist.P2POp(dist.isend, cur[0], nxt, group),
+                   dist.P2POp(dist.isend, cur[1], nxt, group),
+                   dist.P2POp(dist.irecv, dst[0], prv, group),
+                   dist.P2POp(dist.irecv, dst[1], prv, group)]
+            reqs = dist.batch_isend_irecv(ops)
+        if used:
+            partial_fn(q, cur[0], cur[1], o_acc, lse_acc, rope_base, rank * L, src * L,
+                       causal=causal, accumulate=not first, out=out if t == last else None)
+            first = False
+        for r in reqs:
+            r.wait()
+    return out
+
+
+def ring_attention_local(q, k, v, rope_base: float, n_ranks: int, causal: bool = True,
+                         out=None, on_rank=None):
+    """The ring's arithmetic for ``n_ranks`` equal slices of one sequence, every rank's
+    schedule run in turn on this device (no process group, no transfers). The kernel calls
+    and their order are those of `ring_attention` on each rank, so the output equals the
+    distributed result. Use it to validate or time the decomposition on one GPU.
+
+    q [B, Hq, S, D], k, v [B, Hkv, S, D] with S a multiple of n_ranks. ``on_rank(r, phase)``,
+    if given, is called with phase "start" before rank r's calls are enqueued and "end"
+    after them (for example to record CUDA events). Returns out [B, Hq, S, D] bf16.
+    """
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("q [B, Hq, S, D], k and v [B, Hkv, S, D]")
+    B, Hq, S, D = q.shape
+    if S % n_ranks:
+        raise ValueError("the sequence length must be a multiple of n_ranks")
+    L = S // n_ranks
+    # preparation: the slices, and each rank's keys rotated at its own positions (as the
+    # owning rank does before the ring starts)
+    qs = [q[:, :, r * L:(r + 1) * L].contiguous() for r in range(n_ranks)]
+    blocks = [(_lib.rope_attn_rotate(k[:, :, s * L:(s + 1) * L].contiguous(), rope_base, s * L),
+               v[:, :, s * L:(s + 1) * L].contiguous()) for s in range(n_ranks)]
+    outs = [torch.empty_like(qs[r]) for r in range(n_ranks)]
+    o_acc = torch.empty((B, Hq, L, D), dtype=torch.float32, device=q.device)
+    lse_acc = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    # the ring's attention: each rank's blocks in its ring order, merged into its accumulator
+    for r in range(n_ranks):
+        if on_rank:
+            on_rank(r, "start")
+        used = [(t, src) for t, src, u in ring_steps(r, n_ranks, causal) if u]
+        for i, (_, src) in enumerate(used):
+            _lib.rope_attn_fwd_partial(qs[r], blocks[src][0], blocks[src][1], o_acc, lse_acc,
+                                       rope_base, r * L, src * L, causal=causal,
+                                       accumulate=i > 0,
+                                       out=outs[r] if i == len(used) - 1 else None)
+        if on_rank:
+            on_rank(r, "end")
+    return torch.cat(outs, dim=2, out=out) if out is not None else torch.cat(outs, dim=2)
