@@ -16,8 +16,12 @@
  * causal mask key j is visible to query i iff its position is not after the query's.
  *
  * Temporary device memory (the rotated keys and the RoPE table of rope_attn_fwd, the
- * per-split partials of rope_attn_decode) is taken with cudaMallocAsync on `stream` and
- * released with cudaFreeAsync on the same stream before the call returns.
+ * per-split partials of rope_attn_decode) is taken stream-ordered on `stream` from a memory
+ * pool that the library creates on each device at its first call there, and released to it
+ * on the same stream before the call returns. The pool keeps up to 512 MiB cached across
+ * stream synchronisations, so calls after a synchronisation find their workspace ready
+ * (with the device's default pool every synchronisation returned the memory, and the next
+ * call waited to map it again). rope_attn_decode_noalloc takes no memory at all.
  */
 #ifndef ROPEATTN_H_
 #define ROPEATTN_H_

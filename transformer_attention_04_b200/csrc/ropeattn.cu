@@ -70,7 +70,14 @@ struct DeviceState {
   unsigned int* status = nullptr;
   int num_sms = 0;
   bool sm100 = false;
+  cudaMemPool_t pool = nullptr;  // stream-ordered pool of the call workspaces
 };
+
+// The call workspaces (rotated keys, RoPE tables, decode partials) come from a pool owned by
+// the library, one per device, that keeps up to this many bytes cached across stream
+// synchronisations. (The device's default pool returns its memory at every synchronisation,
+// so the first call after each one would map memory again.)
+constexpr unsigned long long kPoolKeepBytes = 512ull << 20;
 constexpr int kMaxDevices = 64;
 DeviceState g_devices[kMaxDevices];
 std::mutex g_devices_mu;
@@ -113,6 +120,19 @@ ra_status device_state(DeviceState** out) {
           (e = set_smem(ra::decode_split_kernel<64>, ra::DecCfg<64>::SMEM)) != cudaSuccess ||
           (e = set_smem(ra::decode_split_kernel<128>, ra::DecCfg<128>::SMEM)) != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    if (st.sm100) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.handleTypes = cudaMemHandleTypeNone;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      if ((e = cudaMemPoolCreate(&st.pool, &props)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemPoolCreate");
+      unsigned long long keep = kPoolKeepBytes;
+      if ((e = cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep)) !=
+          cudaSuccess)
+        return cuda_fail(e, "cudaMemPoolSetAttribute");
     }
     st.ready = true;
   }
@@ -324,8 +344,8 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
   const size_t krot_bytes = cached ? 0 : (kbytes + 255) & ~static_cast<size_t>(255);
   const size_t tab_bytes = static_cast<size_t>(tab_len) * (D / 2) * sizeof(float2);
   void* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, krot_bytes + tab_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, krot_bytes + tab_bytes, ds->pool, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(workspace)");
   void* k_rot = ws;
   float2* tab = reinterpret_cast<float2*>(static_cast<char*>(ws) + krot_bytes);
 
@@ -438,8 +458,8 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   // keys arrive rotated)
   const size_t tab_bytes = static_cast<size_t>(Sq) * (D / 2) * sizeof(float2);
   void* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, tab_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, tab_bytes, ds->pool, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(workspace)");
   float2* tab = static_cast<float2*>(ws);
   ra::rope_table_kernel<<<grid_for(static_cast<long long>(Sq) * (D / 2), 256, ds->num_sms), 256,
                           0, s>>>(tab, a.q_pos0, Sq, D, a.rope_base);
@@ -602,8 +622,8 @@ ra_status decode_impl(const DecodeArgs& a, cudaStream_t s) {
 
   void* ws = scratch;
   if (!a.noalloc) {
-    cudaError_t e = cudaMallocAsync(&ws, po_bytes + pml_bytes, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(decode partials)");
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, po_bytes + pml_bytes, ds->pool, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(decode partials)");
   }
   ra::DecParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
