@@ -267,7 +267,10 @@ RA_API long long rope_attn_set_wait_limit(long long limit);
  * around its split kernel. rope_attn_profile_read(which = 0: prefill attention kernel,
  * 1: decode split kernel) waits for the recorded events, returns the summed kernel time in
  * milliseconds and the number of launches, and starts a new count. Enabling (or disabling)
- * also starts a new count. Meant for one device at a time; not for concurrent callers.
+ * also starts a new count. Enabling creates, on the current device, the event pairs of the
+ * first 1024 launches of each kind (so that profiled calls only record events; more are made
+ * as needed) and returns RA_ERR_CUDA if that fails. Meant for one device at a time; not for
+ * concurrent callers.
  */
 RA_API ra_status rope_attn_profile_enable(int enable);
 RA_API ra_status rope_attn_profile_read(int which, double* total_ms, int* launches);

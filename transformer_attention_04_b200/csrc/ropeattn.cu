@@ -679,6 +679,29 @@ ra_status rope_attn_profile_enable(int enable) {
   std::lock_guard<std::mutex> lock(g_prof_mu);
   g_prof_on = enable != 0;
   g_prof[0].used = g_prof[1].used = 0;
+  if (!g_prof_on) return RA_OK;
+  // create the event pairs of the first kProfReserve launches of each kind now, on the
+  // current device, so that profiled calls only record events
+  constexpr size_t kProfReserve = 1024;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  for (ProfKind& pk : g_prof) {
+    if (pk.device != dev) {
+      for (auto& ev : pk.ev) { cudaEventDestroy(ev.first); cudaEventDestroy(ev.second); }
+      pk.ev.clear();
+      pk.device = dev;
+    }
+    while (pk.ev.size() < kProfReserve) {
+      cudaEvent_t a, b;
+      if ((e = cudaEventCreate(&a)) != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+      if ((e = cudaEventCreate(&b)) != cudaSuccess) {
+        cudaEventDestroy(a);
+        return cuda_fail(e, "cudaEventCreate");
+      }
+      pk.ev.emplace_back(a, b);
+    }
+  }
   return RA_OK;
 }
 
