@@ -14,4 +14,6 @@ from .ref import (  # noqa: F401
     merge_partials,
     ring_shards,
     ring_attention,
+    zigzag_chunks,
+    ring_attention_zigzag,
 )

@@ -71,6 +71,8 @@ __all__ = [
     "merge_partials",
     "ring_shards",
     "ring_attention",
+    "zigzag_chunks",
+    "ring_attention_zigzag",
 ]
 
 
@@ -400,3 +402,49 @@ def ring_attention(q, k, v, rope_base: float, n_ranks: int, causal: bool = True)
         outs.append(o_acc)
         lses.append(lse_acc)
     return np.concatenate(outs, axis=2), np.concatenate(lses, axis=2)
+
+
+def zigzag_chunks(S: int, n: int):
+    """The two position ranges of each of n ranks when one sequence of S positions is cut into
+    2n equal chunks and rank r takes chunks r and 2n-1-r."""
+    if S % (2 * n):
+        raise ValueError("the zig-zag split needs S divisible by 2 * n_ranks")
+    c = S // (2 * n)
+    return [((r * c, (r + 1) * c), ((2 * n - 1 - r) * c, (2 * n - r) * c)) for r in range(n)]
+
+
+def ring_attention_zigzag(q, k, v, rope_base: float, n_ranks: int, causal: bool = True):
+    """Ring attention with the zig-zag split: rank r holds chunks r and 2n-1-r of the
+    sequence, and the blocks passed around the ring are these chunk pairs.
+
+    At step t rank r holds the pair of rank (r - t) mod n. Each of its two query chunks
+    attends each of the pair's two key chunks, except (under the causal mask) a key chunk that
+    lies wholly after the query chunk; every partial result is merged into that query chunk's
+    running result. Returns (o [B, Hq, S, D], lse [B, Hq, S]) in sequence order.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    S = q.shape[2]
+    if k.shape[2] != S:
+        raise ValueError("ring attention here splits one sequence: Sq must equal Sk")
+    chunks = zigzag_chunks(S, n_ranks)
+    k_rot = {rng: rope_rotate(k[:, :, rng[0]:rng[1]], np.arange(*rng), rope_base)
+             for pair in chunks for rng in pair}
+    o = np.zeros(q.shape[:3] + (v.shape[-1],))
+    lse = np.full(q.shape[:3], -np.inf)
+    for r in range(n_ranks):
+        for qa, qb in chunks[r]:
+            o_acc, lse_acc = None, None
+            for t in range(n_ranks):
+                for ka, kb in chunks[(r - t) % n_ranks]:
+                    if causal and ka > qa:
+                        continue  # the key chunk lies wholly after the query chunk
+                    o_p, lse_p = rope_attn_fwd_partial(q[:, :, qa:qb], k_rot[(ka, kb)],
+                                                       v[:, :, ka:kb], rope_base, qa, ka, causal)
+                    if o_acc is None:
+                        o_acc, lse_acc = o_p, lse_p
+                    else:
+                        o_acc, lse_acc = merge_partials(o_acc, lse_acc, o_p, lse_p)
+            o[:, :, qa:qb], lse[:, :, qa:qb] = o_acc, lse_acc
+    return o, lse

@@ -695,3 +695,46 @@ def test_planted_ring_mistakes_are_caught(monkeypatch):
         return o, l - np.max(s, axis=-1) / math.sqrt(D)
     monkeypatch.setattr(ref, "rope_attn_fwd_partial", lse_without_max)
     assert not lse_pin()
+
+
+def test_zigzag_chunks_cover_the_sequence_once():
+    for S, n in ((32, 4), (12, 3), (4, 2), (16, 1)):
+        ch = oracle.zigzag_chunks(S, n)
+        spans = sorted(rng for pair in ch for rng in pair)
+        assert spans[0][0] == 0 and spans[-1][1] == S
+        assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+        # each rank's two chunks are mirror images: their causal work is the same for all ranks
+        assert all(lo[0] + hi[0] == S - (S // (2 * n)) for lo, hi in ch)
+
+
+@pytest.mark.parametrize("S,n", [(40, 1), (40, 2), (36, 3), (64, 4)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_zigzag_ring_equals_full_attention(S, n, causal):
+    rng = np.random.default_rng(88)
+    q = rng.standard_normal((2, 4, S, 8))
+    k = rng.standard_normal((2, 2, S, 8))
+    v = rng.standard_normal((2, 2, S, 8))
+    o, lse = oracle.ring_attention_zigzag(q, k, v, 10000.0, n, causal)
+    np.testing.assert_allclose(o, oracle.rope_attn_fwd(q, k, v, 10000.0, 0, causal),
+                               atol=1e-13, rtol=0)
+    _, want_l = oracle.ring_attention(q, k, v, 10000.0, 1, causal)
+    np.testing.assert_allclose(lse, want_l, atol=1e-13, rtol=0)
+
+
+def test_planted_zigzag_mistakes_are_caught(monkeypatch):
+    rng = np.random.default_rng(89)
+    q, k, v = rng.standard_normal((1, 2, 24, 4)), rng.standard_normal((1, 1, 24, 4)), \
+        rng.standard_normal((1, 1, 24, 4))
+    full = oracle.rope_attn_fwd(q, k, v, 10000.0)
+
+    def pin():
+        return np.allclose(ref.ring_attention_zigzag(q, k, v, 10000.0, 3)[0], full, atol=1e-12)
+
+    assert pin()
+    orig = ref.zigzag_chunks
+    # a rank's second chunk taken at the wrong place (2n-2-r instead of 2n-1-r), so one chunk
+    # is never a key and another is used twice
+    monkeypatch.setattr(ref, "zigzag_chunks", lambda S, n: [
+        (a, ((2 * n - 2 - r) * (S // (2 * n)), (2 * n - 1 - r) * (S // (2 * n))))
+        for r, (a, _) in enumerate(orig(S, n))])
+    assert not pin()
