@@ -478,7 +478,7 @@ PAGE = 16  # the paged row: 16-token pages
 RING_RANKS = 8  # the ring row: the 32k-token workload over 8 ranks (4096 tokens each)
 
 
-def ring_local_timed(ra, Wl, q, k, v, reps: int):
+def ring_local_timed(ra, Wl, q, k, v, reps: int, layout: str = "contiguous"):
     """Time the attention phase of an 8-rank ring run rank after rank on this GPU (every
     rank's partial-attention calls in its ring order; key rotation and slicing excluded).
     Returns (ms per pass, per-rank ms of the last pass)."""
@@ -489,11 +489,12 @@ def ring_local_timed(ra, Wl, q, k, v, reps: int):
         e.record()
         evs[(r, phase)] = e
 
-    ra.ring_attention_local(q, k, v, Wl.rope_base, RING_RANKS, True)
+    ra.ring_attention_local(q, k, v, Wl.rope_base, RING_RANKS, True, layout=layout)
     total, per = 0.0, []
     for _ in range(reps):
         evs.clear()
-        ra.ring_attention_local(q, k, v, Wl.rope_base, RING_RANKS, True, on_rank=hook)
+        ra.ring_attention_local(q, k, v, Wl.rope_base, RING_RANKS, True, on_rank=hook,
+                                layout=layout)
         torch.cuda.synchronize()
         total += evs[(0, "start")].elapsed_time(evs[(RING_RANKS - 1, "end")])
         per = [evs[(r, "start")].elapsed_time(evs[(r, "end")]) for r in range(RING_RANKS)]
@@ -556,6 +557,18 @@ def next_rows_leg(ra, world, rank, dev, peaks):
     e["kernel"] = "attn_fwd_sm100_kernel"
     e["block_traffic"] = recorded_traffic("attn_fwd_sm100_kernel ring")
     res["ring_long_context_8_ranks"] = e
+    # the same ring with the zig-zag split (rank r holds chunks r and 15 - r of 2048 tokens):
+    # every rank attends the same number of chunk blocks
+    ms, per_rank = ring_local_timed(ra, Wl, q, k, v, 3, layout="zigzag")
+    e = _rate_entry(
+        f"{Wl.name} B{Wl.B} Hq{Wl.Hq} Hkv{Wl.Hkv} S{Wl.Sq} D{Wl.D} causal as a {RING_RANKS}-rank "
+        f"zig-zag ring (chunks of {L // 2} tokens, rank r holds chunks r and "
+        f"{2 * RING_RANKS - 1}-r), ranks run in turn on one GPU", ms, Wl.flops(), world,
+        "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s")
+    e["per_rank_ms"] = per_rank
+    e["critical_rank_ms"] = max(per_rank)
+    e["exchange_bytes_per_step"] = 2 * Wl.B * Wl.Hkv * L * Wl.D * 2
+    res["ring_long_context_8_ranks_zigzag"] = e
     del q, k, v, out
     # chunked prefill into a cache: the headline prefill with its keys/values written out
     P = PREFILL_W

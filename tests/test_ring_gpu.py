@@ -146,6 +146,17 @@ def test_ring_on_one_gpu_equals_full_attention(n, causal):
     assert_parity(got, want, f"ring n={n} causal={causal}")
 
 
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("n", [2, 3])
+def test_zigzag_ring_on_one_gpu_equals_full_attention(n, causal):
+    B, Hq, Hkv, S, D, base = 1, 8, 2, 1200, 128, 500000.0
+    q, k, v = _bf16((B, Hq, S, D), 19), _bf16((B, Hkv, S, D), 20), _bf16((B, Hkv, S, D), 21)
+    want = oracle.rope_attn_fwd(to_f64(q), to_f64(k), to_f64(v), base, 0, causal)
+    got = ra.ring_attention_local(q.cuda(), k.cuda(), v.cuda(), base, n, causal, layout="zigzag")
+    _ok()
+    assert_parity(got, want, f"zig-zag ring n={n} causal={causal}")
+
+
 def test_ring_long_context_eight_ranks_sampled_rows():
     # the 32k-token workload as an 8-rank ring (4096 tokens per rank), the decomposition the
     # benchmark times; every checked row is an exact check of that row
@@ -159,6 +170,10 @@ def test_ring_long_context_eight_ranks_sampled_rows():
                                 to_f64(v[:, [h // 8 for h in heads]]), W.rope_base, 0, True,
                                 rows=rows)
     assert_parity(got[:, heads][:, :, rows], want, "8-rank ring, long context")
+    got = ra.ring_attention_local(q.cuda(), k.cuda(), v.cuda(), W.rope_base, 8, True,
+                                  layout="zigzag")
+    _ok()
+    assert_parity(got[:, heads][:, :, rows], want, "8-rank zig-zag ring, long context")
 
 
 def _free_port():

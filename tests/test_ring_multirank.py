@@ -31,7 +31,7 @@ def _inputs(B, Hq, Hkv, S, D, seed):
             g.standard_normal((B, Hkv, S, D)))
 
 
-def _worker(rank, world, port, causal, q_out):
+def _worker(rank, world, port, causal, q_out, layout="contiguous"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import datetime
@@ -66,13 +66,23 @@ def _worker(rank, world, port, causal, q_out):
 
     B, Hq, Hkv, L, D = 1, 4, 2, 6, 8
     q, k, v = _inputs(B, Hq, Hkv, world * L, D, seed=90)
-    sl = slice(rank * L, (rank + 1) * L)
-    res = ring_attention(torch.from_numpy(q[:, :, sl].copy()), torch.from_numpy(k[:, :, sl].copy()),
-                         torch.from_numpy(v[:, :, sl].copy()), 1000.0, causal=causal,
-                         partial_fn=cpu_partial, rotate_fn=cpu_rotate)
+    if layout == "zigzag":
+        c = L // 2
+        cut = lambda x, i: torch.from_numpy(x[:, :, i * c:(i + 1) * c].copy())
+        mine = (rank, 2 * world - 1 - rank)
+        res = ring_attention(tuple(cut(q, i) for i in mine), tuple(cut(k, i) for i in mine),
+                             tuple(cut(v, i) for i in mine), 1000.0, causal=causal,
+                             layout="zigzag", partial_fn=cpu_partial, rotate_fn=cpu_rotate)
+        res = np.stack([res[0].numpy(), res[1].numpy()])
+    else:
+        sl = slice(rank * L, (rank + 1) * L)
+        res = ring_attention(torch.from_numpy(q[:, :, sl].copy()),
+                             torch.from_numpy(k[:, :, sl].copy()),
+                             torch.from_numpy(v[:, :, sl].copy()), 1000.0, causal=causal,
+                             partial_fn=cpu_partial, rotate_fn=cpu_rotate).numpy()
     dist.barrier()
     dist.destroy_process_group()
-    q_out.put((rank, res.numpy(), calls))
+    q_out.put((rank, res, calls))
 
 
 @pytest.mark.parametrize("world", [2, 3])
@@ -120,3 +130,45 @@ def test_ring_steps_schedule():
     for world in (2, 3, 5):
         for r in range(world):
             assert sorted(s for _, s, _ in ring_steps(r, world, False)) == list(range(world))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [True, False])
+def test_zigzag_ring_attention_gloo_equals_full(world, causal):
+    sys.path.insert(0, ROOT)
+    import oracle
+
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q_out = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, causal, q_out, "zigzag"))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted([q_out.get(timeout=180) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    L, c = 6, 3
+    q, k, v = _inputs(1, 4, 2, world * L, 8, seed=90)
+    want = oracle.rope_attn_fwd(q, k, v, 1000.0, 0, causal)
+    n_blocks = []
+    for rank, res, calls in got:
+        for half, chunk in enumerate((rank, 2 * world - 1 - rank)):
+            np.testing.assert_allclose(res[half], want[:, :, chunk * c:(chunk + 1) * c],
+                                       atol=1e-5, rtol=0)
+        n_blocks.append(len(calls))
+        # every call has the query chunk at or after the key chunk under the mask
+        assert all(kp <= qp for qp, kp, _, _ in calls) or not causal
+    # balanced: every rank attends the same number of chunk blocks
+    assert len(set(n_blocks)) == 1
+
+
+def test_zigzag_steps_schedule():
+    sys.path.insert(0, ROOT)
+    from transformer_attention_04_b200.ring import zigzag_steps
+    for world in (1, 2, 3, 4, 8):
+        counts = [len(zigzag_steps(r, world, True)) for r in range(world)]
+        assert counts == [2 * world + 1] * world  # 2 diagonal halves + 2*world - 1 full
+        for r in range(world):
+            assert len(zigzag_steps(r, world, False)) == 4 * world
