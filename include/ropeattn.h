@@ -95,6 +95,15 @@ RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void
  *   causal: key j is allowed to query row i iff k_pos0 + j <= q_pos0 + i; requires
  *   q_pos0 >= k_pos0, so that every row sees at least the block's first key. zero: all keys.
  *   q_pos0, k_pos0 >= 0; q_pos0 + Sq and k_pos0 + Sk at most 2^30.
+ * Views into longer sequences: q_rows, kv_rows and acc_rows are the numbers of rows between
+ * consecutive heads of q, of k_rot and v, and of o_acc / lse_acc / out (0 = packed: Sq, Sk,
+ * Sq; otherwise at least Sq, Sk, Sq). Head (b, h) of q then starts (b*H + h) * q_rows * D
+ * elements after q, and so on. This lets a call read rows [a, a+Sq) of a [B, H, S_alloc, D]
+ * tensor (pointer advanced by a*D elements, rows = S_alloc) and merge into the matching rows
+ * of an accumulator.
+ * Two query segments: with 0 < q_split < Sq, rows i >= q_split sit at q_pos1 + (i - q_split)
+ * instead of q_pos0 + i (two separate slices of one sequence in one launch). Allowed only
+ * with causal == 0. q_split = 0 means one segment.
  * o_acc, lse_acc and out must not overlap the inputs or each other; o_acc is 16-byte
  * aligned, lse_acc 4-byte aligned. D in {64, 128}, Hq % Hkv == 0, sizes >= 1. Runs the
  * prefill kernel of rope_attn_fwd with its fp32 epilogue (one launch, plus the RoPE table of
@@ -105,7 +114,8 @@ RA_API ra_status rope_attn_fwd_partial(const void* q, const void* k_rot, const v
                                        float* o_acc, float* lse_acc, void* out, int B, int Hq,
                                        int Hkv, int Sq, int Sk, int D, float rope_base,
                                        int q_pos0, int k_pos0, int causal, int accumulate,
-                                       ra_stream_t stream);
+                                       int q_rows, int kv_rows, int acc_rows, int q_split,
+                                       int q_pos1, ra_stream_t stream);
 
 /*
  * Prefill with a sliding window and/or straight into a KV cache (chunked prefill).
@@ -147,6 +157,17 @@ RA_API ra_status rope_attn_prefill(const void* q, const void* k, const void* v, 
  */
 RA_API ra_status rope_attn_rotate(const void* x, void* x_rot, int B, int H, int S, int D,
                            float rope_base, int pos_offset, ra_stream_t stream);
+
+/*
+ * rope_attn_rotate on views into longer sequences: x_rows and out_rows are the numbers of rows
+ * between consecutive heads of x and of x_rot (0 = S, packed; otherwise at least S). This
+ * rotates rows [a, a+S) of a [B, H, S_alloc, D] tensor in place, or into the matching rows of
+ * another, at positions pos_offset + s. In place (x == x_rot) requires x_rows == out_rows;
+ * otherwise the two extents must not overlap. Other arguments and errors as rope_attn_rotate.
+ */
+RA_API ra_status rope_attn_rotate_rows(const void* x, void* x_rot, int B, int H, int S, int D,
+                                       float rope_base, int pos_offset, int x_rows, int out_rows,
+                                       ra_stream_t stream);
 
 /*
  * One decode step over a pre-rotated KV cache (split-KV with a log-sum-exp combine).

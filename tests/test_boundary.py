@@ -222,9 +222,9 @@ def test_decode_paged_rejects(lib, kw):
 
 def partial(lib, q=FAKE, k=FAKE + (1 << 40), v=FAKE + (2 << 40), o=FAKE + (3 << 40),
             lse=FAKE + (4 << 40), out=0, B=1, Hq=4, Hkv=2, Sq=16, Sk=16, D=64, base=10000.0,
-            qp=32, kp=16, causal=1, acc=0):
+            qp=32, kp=16, causal=1, acc=0, q_rows=0, kv_rows=0, acc_rows=0, split=0, qp1=0):
     return lib.rope_attn_fwd_partial(q, k, v, o, lse, out, B, Hq, Hkv, Sq, Sk, D, base, qp, kp,
-                                     causal, acc, None)
+                                     causal, acc, q_rows, kv_rows, acc_rows, split, qp1, None)
 
 
 @pytest.mark.parametrize("kw,want", [
@@ -240,6 +240,14 @@ def partial(lib, q=FAKE, k=FAKE + (1 << 40), v=FAKE + (2 << 40), o=FAKE + (3 << 
     (dict(lse=FAKE + (3 << 40)), ra.RA_ERR_INVALID_ARG),  # lse_acc overlaps o_acc
     (dict(out=FAKE + (2 << 40)), ra.RA_ERR_INVALID_ARG),  # out overlaps v
     (dict(D=96), ra.RA_ERR_UNSUPPORTED),
+    (dict(q_rows=15), ra.RA_ERR_INVALID_ARG),           # head stride shorter than the rows
+    (dict(kv_rows=-1), ra.RA_ERR_INVALID_ARG),
+    (dict(acc_rows=8), ra.RA_ERR_INVALID_ARG),
+    (dict(split=8, qp1=100), ra.RA_ERR_INVALID_ARG),    # two query segments need causal == 0
+    (dict(split=8, qp1=-1, causal=0), ra.RA_ERR_INVALID_ARG),
+    (dict(split=-1), ra.RA_ERR_INVALID_ARG),
+    # o_acc inside k's strided extent (2 heads 64 rows apart: 80 rows of 128 bytes)
+    (dict(kv_rows=64, o=FAKE + (1 << 40) + 8192), ra.RA_ERR_INVALID_ARG),
 ])
 def test_partial_rejects(lib, kw, want):
     assert partial(lib, **kw) == want

@@ -222,3 +222,67 @@ def test_partial_guards():
         assert bool((g[:GUARD] == 0x5A5A5A5A).all()) and bool((g[GUARD + n:] == 0x5A5A5A5A).all())
     assert not bool(torch.isnan(o_acc).any()) and not bool(torch.isnan(lse).any())
     assert torch.equal(q0, qc) and torch.equal(kr0, krc) and torch.equal(v0, vc)
+
+
+def test_partial_on_views_of_longer_tensors():
+    # q rows [40, 240) of a 400-row tensor, keys rows [100, 400) of a 512-row tensor, the
+    # accumulator rows [40, 240) of a 400-row one: each call reads and writes only its rows
+    B, Hq, Hkv, D, base = 2, 4, 2, 128, 10000.0
+    qa, qb, ka, kb = 40, 240, 100, 400
+    q_full = _bf16((B, Hq, 400, D), 22)
+    k_full, v_full = _bf16((B, Hkv, 512, D), 23), _bf16((B, Hkv, 512, D), 24)
+    kr_full = _rotated_keys(k_full, -ka + 700, base)  # row j rotated at 700 + (j - ka)
+    q_pos0, k_pos0 = 900, 700
+    want_o, want_l = oracle.rope_attn_fwd_partial(
+        to_f64(q_full[:, :, qa:qb]), to_f64(kr_full[:, :, ka:kb]), to_f64(v_full[:, :, ka:kb]),
+        base, q_pos0, k_pos0, True)
+    qg, krg, vg = q_full.cuda(), kr_full.cuda(), v_full.cuda()
+    acc_o = torch.full((B, Hq, 400, D), 7.0, device="cuda")
+    acc_l = torch.full((B, Hq, 400), 7.0, device="cuda")
+    out = torch.full((B, Hq, 400, D), 7.0, device="cuda", dtype=torch.bfloat16)
+    ra.rope_attn_fwd_partial(qg[:, :, qa:qb], krg[:, :, ka:kb], vg[:, :, ka:kb],
+                             acc_o[:, :, qa:qb], acc_l[:, :, qa:qb], base, q_pos0, k_pos0, True,
+                             out=out[:, :, qa:qb])
+    _ok()
+    assert_parity(acc_o[:, :, qa:qb], want_o, "o_acc view")
+    assert_parity(out[:, :, qa:qb], want_o, "out view")
+    _check_lse(acc_l[:, :, qa:qb], want_l, "lse view")
+    # rows outside the view are untouched
+    for t in (acc_o, acc_l, out.float()):
+        assert bool((t[:, :, :qa] == 7.0).all()) and bool((t[:, :, qb:] == 7.0).all())
+
+
+def test_partial_two_query_segments():
+    # rows [0, 256) at positions 3000.., rows [256, 400) at 100.. against keys at 5000..
+    # (unmasked: two slices of one sequence in one launch)
+    B, Hq, Hkv, Sq, Sk, D, base = 1, 8, 2, 400, 300, 64, 500000.0
+    split, p0, p1, kp = 256, 3000, 100, 5000
+    q, k, v = _bf16((B, Hq, Sq, D), 25), _bf16((B, Hkv, Sk, D), 26), _bf16((B, Hkv, Sk, D), 27)
+    kr = _rotated_keys(k, kp, base)
+    a = oracle.rope_attn_fwd_partial(to_f64(q[:, :, :split]), to_f64(kr), to_f64(v), base, p0,
+                                     kp, False)
+    b = oracle.rope_attn_fwd_partial(to_f64(q[:, :, split:]), to_f64(kr), to_f64(v), base, p1,
+                                     kp, False)
+    want_o = np.concatenate([a[0], b[0]], axis=2)
+    want_l = np.concatenate([a[1], b[1]], axis=2)
+    o_acc = torch.empty((B, Hq, Sq, D), device="cuda")
+    lse = torch.empty((B, Hq, Sq), device="cuda")
+    ra.rope_attn_fwd_partial(q.cuda(), kr.cuda(), v.cuda(), o_acc, lse, base, p0, kp, False,
+                             q_split=split, q_pos1=p1)
+    _ok()
+    assert_parity(o_acc, want_o, "two segments")
+    _check_lse(lse, want_l, "two segments")
+
+
+def test_rotate_views():
+    # rotate rows [30, 130) of one tensor into rows [10, 110) of another at positions 500..
+    x = _bf16((2, 3, 160, 64), 28)
+    xg = x.cuda()
+    out = torch.zeros((2, 3, 200, 64), device="cuda", dtype=torch.bfloat16)
+    ra.rope_attn_rotate(xg[:, :, 30:130], 10000.0, 500, out=out[:, :, 10:110])
+    _ok()
+    want = oracle.rope_rotate(to_f64(x[:, :, 30:130]), 500 + np.arange(100), 10000.0)
+    got = out[:, :, 10:110].double().cpu().numpy()
+    # one bf16 rounding of values of magnitude up to ~4
+    assert np.max(np.abs(got - want)) <= 2 ** -7 * max(1.0, np.max(np.abs(want)))
+    assert bool((out[:, :, :10] == 0).all()) and bool((out[:, :, 110:] == 0).all())

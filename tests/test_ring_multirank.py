@@ -51,10 +51,20 @@ def _worker(rank, world, port, causal, q_out, layout="contiguous"):
         return out
 
     def cpu_partial(q, k_rot, v, o_acc, lse_acc, rope_base, q_pos0, k_pos0, causal=True,
-                    accumulate=False, out=None):
+                    accumulate=False, out=None, q_split=0, q_pos1=0):
         calls.append((q_pos0, k_pos0, bool(accumulate), out is not None))
-        o, lse = oracle.rope_attn_fwd_partial(q.numpy(), k_rot.numpy(), v.numpy(), rope_base,
-                                              q_pos0, k_pos0, causal)
+        if 0 < q_split < q.shape[2]:
+            # two query segments (unmasked): each row's result depends only on its position
+            assert not causal
+            parts = [oracle.rope_attn_fwd_partial(q[:, :, :q_split].numpy(), k_rot.numpy(),
+                                                  v.numpy(), rope_base, q_pos0, k_pos0, False),
+                     oracle.rope_attn_fwd_partial(q[:, :, q_split:].numpy(), k_rot.numpy(),
+                                                  v.numpy(), rope_base, q_pos1, k_pos0, False)]
+            o = np.concatenate([parts[0][0], parts[1][0]], axis=2)
+            lse = np.concatenate([parts[0][1], parts[1][1]], axis=2)
+        else:
+            o, lse = oracle.rope_attn_fwd_partial(q.numpy(), k_rot.numpy(), v.numpy(),
+                                                  rope_base, q_pos0, k_pos0, causal)
         if accumulate:
             o, lse = oracle.merge_partials(o_acc.double().numpy(), lse_acc.double().numpy(), o,
                                            lse)
@@ -68,12 +78,12 @@ def _worker(rank, world, port, causal, q_out, layout="contiguous"):
     q, k, v = _inputs(B, Hq, Hkv, world * L, D, seed=90)
     if layout == "zigzag":
         c = L // 2
-        cut = lambda x, i: torch.from_numpy(x[:, :, i * c:(i + 1) * c].copy())
         mine = (rank, 2 * world - 1 - rank)
-        res = ring_attention(tuple(cut(q, i) for i in mine), tuple(cut(k, i) for i in mine),
-                             tuple(cut(v, i) for i in mine), 1000.0, causal=causal,
+        local = lambda x: torch.from_numpy(
+            np.concatenate([x[:, :, i * c:(i + 1) * c] for i in mine], axis=2))
+        res = ring_attention(local(q), local(k), local(v), 1000.0, causal=causal,
                              layout="zigzag", partial_fn=cpu_partial, rotate_fn=cpu_rotate)
-        res = np.stack([res[0].numpy(), res[1].numpy()])
+        res = np.stack([res[:, :, :c].numpy(), res[:, :, c:].numpy()])
     else:
         sl = slice(rank * L, (rank + 1) * L)
         res = ring_attention(torch.from_numpy(q[:, :, sl].copy()),
@@ -152,23 +162,36 @@ def test_zigzag_ring_attention_gloo_equals_full(world, causal):
     L, c = 6, 3
     q, k, v = _inputs(1, 4, 2, world * L, 8, seed=90)
     want = oracle.rope_attn_fwd(q, k, v, 1000.0, 0, causal)
-    n_blocks = []
+    n_calls = []
     for rank, res, calls in got:
         for half, chunk in enumerate((rank, 2 * world - 1 - rank)):
             np.testing.assert_allclose(res[half], want[:, :, chunk * c:(chunk + 1) * c],
                                        atol=1e-5, rtol=0)
-        n_blocks.append(len(calls))
-        # every call has the query chunk at or after the key chunk under the mask
-        assert all(kp <= qp for qp, kp, _, _ in calls) or not causal
-    # balanced: every rank attends the same number of chunk blocks
-    assert len(set(n_blocks)) == 1
+        n_calls.append(len(calls))
+        # the first call of the rank overwrites, the last one writes the output
+        assert not calls[0][2] and calls[-1][3]
+    # balanced: every rank makes the same launches (world + 2 masked, world unmasked)
+    assert n_calls == [world + 2 if causal else world] * world
 
 
-def test_zigzag_steps_schedule():
+def test_zigzag_calls_schedule():
     sys.path.insert(0, ROOT)
-    from transformer_attention_04_b200.ring import zigzag_steps
+    from transformer_attention_04_b200.ring import zigzag_calls
+    size = {"lo": 1, "hi": 1, "all": 2}
     for world in (1, 2, 3, 4, 8):
-        counts = [len(zigzag_steps(r, world, True)) for r in range(world)]
-        assert counts == [2 * world + 1] * world  # 2 diagonal halves + 2*world - 1 full
         for r in range(world):
-            assert len(zigzag_steps(r, world, False)) == 4 * world
+            calls = zigzag_calls(r, world, True)
+            assert len(calls) == world + 2
+            # chunk blocks attended (a masked diagonal one counts half): 2*world on every rank
+            work = sum(size[qh] * size[kh] * (0.5 if m else 1) for _, _, qh, kh, m in calls)
+            assert work == 2 * world
+            # every (query chunk, key chunk) pair with the key chunk not after the query chunk
+            # is attended exactly once
+            chunk = lambda owner, h: owner if h == "lo" else 2 * world - 1 - owner
+            halves = {"lo": ["lo"], "hi": ["hi"], "all": ["lo", "hi"]}
+            seen = sorted((chunk(r, a), chunk(s, b)) for _, s, qh, kh, _ in calls
+                          for a in halves[qh] for b in halves[kh])
+            want = sorted((qc, kc) for qc in (chunk(r, "lo"), chunk(r, "hi"))
+                          for kc in range(2 * world) if kc <= qc)
+            assert seen == want
+            assert len(zigzag_calls(r, world, False)) == world

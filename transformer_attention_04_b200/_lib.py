@@ -24,8 +24,9 @@ SIGNATURES = {
     "rope_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
                                _P]),
     "rope_attn_rotate": (_I, [_P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "rope_attn_rotate_rows": (_I, [_P, _P, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "rope_attn_fwd_partial": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
-                                   _I, _P]),
+                                   _I, _I, _I, _I, _I, _I, _P]),
     "rope_attn_decode": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "rope_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "rope_attn_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I,
@@ -141,32 +142,54 @@ def rope_attn_prefill(q, k, v, rope_base: float, pos_offset: int = 0, causal: bo
     return out
 
 
+def _head_rows(t, name, dtype, shape):
+    """Rows between consecutive heads of a [B, H, S(, D)] view whose rows are packed (a slice
+    along S of a longer tensor is allowed); checks dtype, device, shape and layout."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != dtype:
+        raise ValueError(f"{name} must be a {dtype} CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    B, H, S = shape[:3]
+    row = shape[3] if len(shape) == 4 else 1
+    st = t.stride()
+    if (len(shape) == 4 and st[3] != 1) or st[2] != row:
+        raise ValueError(f"{name}: rows must be packed along the last axis")
+    rows = st[1] // row if H > 1 else (st[0] // row if B > 1 else S)
+    if st[1] % row or rows < S or (B > 1 and st[0] != H * rows * row):
+        raise ValueError(f"{name}: heads must be evenly spaced slices of >= {S} rows")
+    return rows
+
+
 def rope_attn_fwd_partial(q, k_rot, v, o_acc, lse_acc, rope_base: float, q_pos0: int,
                           k_pos0: int, causal: bool = True, accumulate: bool = False, out=None,
-                          stream=None):
-    """One ring-attention block: q [B,Hq,Sq,D] (rotated here to q_pos0+i) against keys k_rot
+                          q_split: int = 0, q_pos1: int = 0, stream=None):
+    """One ring-attention block: q [B,Hq,Sq,D] (rotated here to q_pos0+i; rows >= q_split at
+    q_pos1 + (i - q_split) when 0 < q_split < Sq, unmasked calls only) against keys k_rot
     [B,Hkv,Sk,D] already rotated to k_pos0+j, and v. The block's normalised output and
     natural-log LSE go to o_acc [B,Hq,Sq,D] / lse_acc [B,Hq,Sq] (fp32), merged with their
-    contents when ``accumulate``; ``out`` (bf16), if given, also receives the merged result."""
-    _check(q, "q")
+    contents when ``accumulate``; ``out`` (bf16), if given, also receives the merged result.
+    Every tensor may be a slice along the sequence axis of a longer one (q[:, :, a:b])."""
     if q.dim() != 4 or k_rot.dim() != 4:
         raise ValueError("q, k_rot, v must be 4-D [B, H, S, D]")
     B, Hq, Sq, D = q.shape
     Hkv, Sk = k_rot.shape[1], k_rot.shape[2]
-    _check(k_rot, "k_rot", (B, Hkv, Sk, D))
-    _check(v, "v", (B, Hkv, Sk, D))
-    for t, name, shape in ((o_acc, "o_acc", (B, Hq, Sq, D)), (lse_acc, "lse_acc", (B, Hq, Sq))):
-        if (not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or
-                not t.is_contiguous() or tuple(t.shape) != shape):
-            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of shape {shape}")
+    q_rows = _head_rows(q, "q", torch.bfloat16, (B, Hq, Sq, D))
+    kv_rows = _head_rows(k_rot, "k_rot", torch.bfloat16, (B, Hkv, Sk, D))
+    if _head_rows(v, "v", torch.bfloat16, (B, Hkv, Sk, D)) != kv_rows:
+        raise ValueError("k_rot and v must have the same layout")
+    acc_rows = _head_rows(o_acc, "o_acc", torch.float32, (B, Hq, Sq, D))
+    if _head_rows(lse_acc, "lse_acc", torch.float32, (B, Hq, Sq)) != acc_rows:
+        raise ValueError("o_acc and lse_acc must have the same row layout")
     o = 0
     if out is not None:
-        _check(out, "out", q.shape)
+        if _head_rows(out, "out", torch.bfloat16, (B, Hq, Sq, D)) != acc_rows:
+            raise ValueError("out must have the row layout of o_acc")
         o = out.data_ptr()
     st = lib().rope_attn_fwd_partial(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(),
                                      o_acc.data_ptr(), lse_acc.data_ptr(), o, B, Hq, Hkv, Sq, Sk,
                                      D, float(rope_base), int(q_pos0), int(k_pos0),
-                                     int(bool(causal)), int(bool(accumulate)), _stream(stream))
+                                     int(bool(causal)), int(bool(accumulate)), q_rows, kv_rows,
+                                     acc_rows, int(q_split), int(q_pos1), _stream(stream))
     _raise(st, "rope_attn_fwd_partial")
     return out
 
@@ -246,14 +269,17 @@ def rope_attn_decode_paged(q, k_pool_rot, v_pool, block_table, pos, max_pos: int
 
 
 def rope_attn_rotate(x, rope_base: float, pos_offset: int = 0, out=None, stream=None):
-    """RoPE-rotate x [B,H,S,D] at positions pos_offset + s; out may be x (in place)."""
-    _check(x, "x")
+    """RoPE-rotate x [B,H,S,D] at positions pos_offset + s; out may be x (in place). x and out
+    may be slices along the sequence axis of longer tensors (x[:, :, a:b])."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 4:
+        raise ValueError("x must be a 4-D [B, H, S, D] tensor")
     B, H, S, D = x.shape
+    x_rows = _head_rows(x, "x", torch.bfloat16, (B, H, S, D))
     if out is None:
-        out = torch.empty_like(x)
-    _check(out, "out", x.shape)
-    st = lib().rope_attn_rotate(x.data_ptr(), out.data_ptr(), B, H, S, D, float(rope_base),
-                                int(pos_offset), _stream(stream))
+        out = torch.empty_like(x, memory_format=torch.contiguous_format)
+    out_rows = _head_rows(out, "out", torch.bfloat16, (B, H, S, D))
+    st = lib().rope_attn_rotate_rows(x.data_ptr(), out.data_ptr(), B, H, S, D, float(rope_base),
+                                     int(pos_offset), x_rows, out_rows, _stream(stream))
     _raise(st, "rope_attn_rotate")
     return out
 

@@ -74,6 +74,7 @@ struct FwdParams {
   float* o_acc;
   float* lse_acc;
   int accumulate;
+  int acc_rows;  // partial mode: rows between heads in o_acc / lse_acc / out (>= Sq)
 };
 
 template <int D>
@@ -536,7 +537,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (p.o_acc != nullptr) {
       if (ok && mbar_wait_warp(bar(C::B_OFULL + s), 0, lim, abort_flag, p.status)) {
         tc_fence_after();
-        const long long row = static_cast<long long>(b * p.Hq + h0 + s) * p.Sq + qrow;
+        const long long row = static_cast<long long>(b * p.Hq + h0 + s) * p.acc_rows + qrow;
         const float lse_new = (m + log2f(l)) * kLn2;
         float w_old = 0.f, w_new = 1.0f / l, lse_out = lse_new;
         if (p.accumulate && qrow < p.Sq) {

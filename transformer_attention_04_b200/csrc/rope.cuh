@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* __restric
                                                           const float2* __restrict__ tab,
                                                           long long nrows_total, int S, int D,
                                                           long long pos0, int tab_off,
-                                                          float base) {
+                                                          float base, int x_rows, int y_rows) {
+  // x_rows / y_rows: rows between consecutive heads of x and y (S when packed)
   const int cpr = D / 8;  // 16-byte chunks per row
   const long long n = nrows_total * cpr;
   const double log2_base = kTable ? 0.0 : log2(static_cast<double>(base));
@@ -70,8 +71,10 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* __restric
        e += (long long)gridDim.x * blockDim.x) {
     const long long row = e / cpr;
     const int chunk = static_cast<int>(e - row * cpr);
-    const int s = static_cast<int>(row % S);
-    const uint4 v = __ldg(x + e);
+    const long long bh = row / S;
+    const int s = static_cast<int>(row - bh * S);
+    const long long xi = (bh * x_rows + s) * cpr + chunk, yi = (bh * y_rows + s) * cpr + chunk;
+    const uint4 v = __ldg(x + xi);
     float2 cs[4];
     if (kTable) {
       const float4* t4 =
@@ -85,7 +88,7 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* __restric
 #pragma unroll
       for (int t = 0; t < 4; ++t) rope_cos_sin(pos0 + s, chunk * 4 + t, D, log2_base, cs[t].x, cs[t].y);
     }
-    y[e] = rotate8(v, cs);
+    y[yi] = rotate8(v, cs);
   }
 }
 

@@ -362,7 +362,7 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
   else
     ra::rope_rotate_kernel<true><<<grid_for(krows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
         static_cast<const uint4*>(a.k), static_cast<uint4*>(k_rot), tab, krows, Sk, D, 0, -tab_lo,
-        a.rope_base);
+        a.rope_base, Sk, Sk);
 
   CUtensorMap tq, tk, tv;
   const long long bkv = static_cast<long long>(B) * Hkv;
@@ -392,6 +392,7 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.o_acc = nullptr;
     p.lse_acc = nullptr;
     p.accumulate = 0;
+    p.acc_rows = Sq;
     rs = launch_attn(p, tq, tk, tv, D, n_units, s);
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
@@ -412,10 +413,23 @@ struct PartialArgs {
   int q_pos0, k_pos0;
   int causal;
   int accumulate;
+  int q_rows, kv_rows, acc_rows;  // rows between consecutive heads (0: packed)
+  int q_split, q_pos1;            // rows >= q_split sit at q_pos1 + (i - q_split)
 };
 
 ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   const int B = a.B, Hq = a.Hq, Hkv = a.Hkv, Sq = a.Sq, Sk = a.Sk, D = a.D;
+  if (a.q_rows < 0 || a.kv_rows < 0 || a.acc_rows < 0) return RA_ERR_INVALID_ARG;
+  const int q_rows = a.q_rows ? a.q_rows : Sq;
+  const int kv_rows = a.kv_rows ? a.kv_rows : Sk;
+  const int acc_rows = a.acc_rows ? a.acc_rows : Sq;
+  if (q_rows < Sq || kv_rows < Sk || acc_rows < Sq) return RA_ERR_INVALID_ARG;
+  // a second query segment: only without the mask (the kernel's causal offset is per launch)
+  const bool two_seg = a.q_split > 0 && a.q_split < Sq;
+  if (a.q_split < 0 || (two_seg && (a.causal || a.q_pos1 < 0 ||
+                                    static_cast<long long>(a.q_pos1) + (Sq - a.q_split) >
+                                        (1LL << 30))))
+    return RA_ERR_INVALID_ARG;
   if (!a.q || !a.k_rot || !a.v || !a.o_acc || !a.lse_acc) return RA_ERR_INVALID_ARG;
   if (!aligned16(a.q) || !aligned16(a.k_rot) || !aligned16(a.v) || !aligned16(a.o_acc) ||
       (reinterpret_cast<uintptr_t>(a.lse_acc) & 3u) || (a.out && !aligned16(a.out)))
@@ -430,19 +444,26 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   // under the causal mask every query row must see the block's first key
   if (a.causal && a.q_pos0 < a.k_pos0) return RA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
-  const size_t qbytes = static_cast<size_t>(B) * Hq * Sq * D * 2;
-  const size_t kbytes = static_cast<size_t>(B) * Hkv * Sk * D * 2;
-  const size_t obytes = static_cast<size_t>(B) * Hq * Sq * D * 4;
-  const size_t lbytes = static_cast<size_t>(B) * Hq * Sq * 4;
+  // extents of the strided views: (heads - 1) full strides plus the last head's rows
+  auto extent = [](long long heads, long long rows, long long used, long long row_bytes) {
+    return static_cast<size_t>(((heads - 1) * rows + used) * row_bytes);
+  };
+  const long long bhq = static_cast<long long>(B) * Hq, bhk = static_cast<long long>(B) * Hkv;
+  const size_t qbytes = extent(bhq, q_rows, Sq, 2LL * D);
+  const size_t kbytes = extent(bhk, kv_rows, Sk, 2LL * D);
+  const size_t obytes = extent(bhq, acc_rows, Sq, 4LL * D);
+  const size_t lbytes = extent(bhq, acc_rows, Sq, 4);
+  const size_t outbytes = extent(bhq, acc_rows, Sq, 2LL * D);
   for (const auto& w : {std::make_pair(static_cast<const void*>(a.o_acc), obytes),
                         std::make_pair(static_cast<const void*>(a.lse_acc), lbytes),
-                        std::make_pair(static_cast<const void*>(a.out), a.out ? qbytes : 0)})
+                        std::make_pair(static_cast<const void*>(a.out), a.out ? outbytes : 0)})
     if (w.second && (overlap(w.first, w.second, a.q, qbytes) ||
                      overlap(w.first, w.second, a.k_rot, kbytes) ||
                      overlap(w.first, w.second, a.v, kbytes)))
       return RA_ERR_INVALID_ARG;
   if (overlap(a.o_acc, obytes, a.lse_acc, lbytes) ||
-      (a.out && (overlap(a.out, qbytes, a.o_acc, obytes) || overlap(a.out, qbytes, a.lse_acc, lbytes))))
+      (a.out && (overlap(a.out, outbytes, a.o_acc, obytes) ||
+                 overlap(a.out, outbytes, a.lse_acc, lbytes))))
     return RA_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
   const int n_slots = (G % 2 == 0) ? 2 : 1;
@@ -454,20 +475,24 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   DeviceState* ds = nullptr;
   ra_status rs = device_state(&ds);
   if (rs != RA_OK) return rs;
-  // workspace: the (cos, sin) table of the query positions q_pos0 .. q_pos0 + Sq - 1 (the
-  // keys arrive rotated)
+  // workspace: the (cos, sin) table of the query rows' positions, one table row per query
+  // row (the keys arrive rotated)
   const size_t tab_bytes = static_cast<size_t>(Sq) * (D / 2) * sizeof(float2);
   void* ws = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(&ws, tab_bytes, ds->pool, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(workspace)");
   float2* tab = static_cast<float2*>(ws);
-  ra::rope_table_kernel<<<grid_for(static_cast<long long>(Sq) * (D / 2), 256, ds->num_sms), 256,
-                          0, s>>>(tab, a.q_pos0, Sq, D, a.rope_base);
+  const int n0 = two_seg ? a.q_split : Sq;
+  ra::rope_table_kernel<<<grid_for(static_cast<long long>(n0) * (D / 2), 256, ds->num_sms), 256,
+                          0, s>>>(tab, a.q_pos0, n0, D, a.rope_base);
+  if (two_seg)
+    ra::rope_table_kernel<<<grid_for(static_cast<long long>(Sq - n0) * (D / 2), 256,
+                                     ds->num_sms), 256, 0, s>>>(
+        tab + static_cast<size_t>(n0) * (D / 2), a.q_pos1, Sq - n0, D, a.rope_base);
   CUtensorMap tq, tk, tv;
-  const long long bkv = static_cast<long long>(B) * Hkv;
-  rs = make_map(&tq, a.q, D, Sq, static_cast<long long>(B) * Hq, 128);
-  if (rs == RA_OK) rs = make_map(&tk, a.k_rot, D, Sk, bkv, 128);
-  if (rs == RA_OK) rs = make_map(&tv, a.v, D, Sk, bkv, 128);
+  rs = make_map(&tq, a.q, D, Sq, bhq, 128, q_rows);
+  if (rs == RA_OK) rs = make_map(&tk, a.k_rot, D, Sk, bhk, 128, kv_rows);
+  if (rs == RA_OK) rs = make_map(&tv, a.v, D, Sk, bhk, 128, kv_rows);
   if (rs == RA_OK) {
     ra::FwdParams p;
     p.out = static_cast<__nv_bfloat16*>(a.out);
@@ -487,6 +512,7 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
     p.o_acc = a.o_acc;
     p.lse_acc = a.lse_acc;
     p.accumulate = a.accumulate ? 1 : 0;
+    p.acc_rows = acc_rows;
     rs = launch_attn(p, tq, tk, tv, D, n_units, s);
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
@@ -768,24 +794,37 @@ ra_status rope_attn_get_device_status(ra_stream_t stream) {
   return (v & ra::kStatusTimeout) ? RA_ERR_DEVICE_TIMEOUT : RA_OK;
 }
 
-ra_status rope_attn_rotate(const void* x, void* x_rot, int B, int H, int S, int D,
-                           float rope_base, int pos_offset, ra_stream_t stream) {
+ra_status rope_attn_rotate_rows(const void* x, void* x_rot, int B, int H, int S, int D,
+                                float rope_base, int pos_offset, int x_rows, int out_rows,
+                                ra_stream_t stream) {
   if (!x || !x_rot || !aligned16(x) || !aligned16(x_rot)) return RA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || S < 1 || D < 8 || D > 256 || D % 8) return RA_ERR_INVALID_ARG;
   if (!(rope_base > 0.f) || !std::isfinite(rope_base) || pos_offset < 0) return RA_ERR_INVALID_ARG;
   if (static_cast<long long>(pos_offset) + S > 0x7fffffffLL) return RA_ERR_INVALID_ARG;
+  if (x_rows < 0 || out_rows < 0) return RA_ERR_INVALID_ARG;
+  if (x_rows == 0) x_rows = S;
+  if (out_rows == 0) out_rows = S;
+  if (x_rows < S || out_rows < S) return RA_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(B) * H * S;
-  const size_t bytes = static_cast<size_t>(rows) * D * 2;
-  if (x != x_rot && overlap(x, bytes, x_rot, bytes)) return RA_ERR_INVALID_ARG;
+  const long long heads = static_cast<long long>(B) * H;
+  const size_t xbytes = static_cast<size_t>((heads - 1) * x_rows + S) * D * 2;
+  const size_t ybytes = static_cast<size_t>((heads - 1) * out_rows + S) * D * 2;
+  // in place only with the same layout; otherwise the two must not share memory
+  if (x == x_rot ? x_rows != out_rows : overlap(x, xbytes, x_rot, ybytes)) return RA_ERR_INVALID_ARG;
   DeviceState* ds = nullptr;
   ra_status rs = device_state(&ds);
   if (rs != RA_OK) return rs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   ra::rope_rotate_kernel<false><<<grid_for(rows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
       static_cast<const uint4*>(x), static_cast<uint4*>(x_rot), nullptr, rows, S, D, pos_offset,
-      0, rope_base);
+      0, rope_base, x_rows, out_rows);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "rope_rotate launch");
+}
+
+ra_status rope_attn_rotate(const void* x, void* x_rot, int B, int H, int S, int D,
+                           float rope_base, int pos_offset, ra_stream_t stream) {
+  return rope_attn_rotate_rows(x, x_rot, B, H, S, D, rope_base, pos_offset, S, S, stream);
 }
 
 
@@ -800,9 +839,10 @@ ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void* out, 
 ra_status rope_attn_fwd_partial(const void* q, const void* k_rot, const void* v, float* o_acc,
                                 float* lse_acc, void* out, int B, int Hq, int Hkv, int Sq, int Sk,
                                 int D, float rope_base, int q_pos0, int k_pos0, int causal,
-                                int accumulate, ra_stream_t stream) {
+                                int accumulate, int q_rows, int kv_rows, int acc_rows,
+                                int q_split, int q_pos1, ra_stream_t stream) {
   PartialArgs a{q, k_rot, v, o_acc, lse_acc, out, B, Hq, Hkv, Sq, Sk, D, rope_base,
-                q_pos0, k_pos0, causal, accumulate};
+                q_pos0, k_pos0, causal, accumulate, q_rows, kv_rows, acc_rows, q_split, q_pos1};
   return partial_impl(a, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -37,24 +37,58 @@ def ring_steps(rank: int, world: int, causal: bool):
     return out
 
 
-def zigzag_steps(rank: int, world: int, causal: bool):
-    """The zig-zag schedule of one rank: the sequence is cut into 2*world equal chunks and
-    rank r holds chunks r and 2*world-1-r (its pair). At step t it holds the pair of rank
-    src = (rank - t) mod world. Returns the (step, src, query half, key half) of every block
-    attended, in order; half 0 is the pair's first chunk, half 1 its second. Under the causal
-    mask a key chunk that lies wholly after the query chunk is skipped; the two chunks of a
-    pair are mirror images, so every rank attends the same number of chunk blocks."""
-    def chunk(owner, half):
-        return owner if half == 0 else 2 * world - 1 - owner
+def zigzag_calls(rank: int, world: int, causal: bool):
+    """The kernel calls of one rank under the zig-zag split.
 
-    out = []
+    The sequence is cut into 2*world chunks of c tokens; rank r holds chunk r then chunk
+    2*world-1-r in one [.., 2c, ..] tensor ("lo" and "hi" halves). At step t it holds the
+    keys/values of rank src = (rank - t) mod world in the same layout. Returns, in order,
+    (step, src, query half, key half, masked) with halves "lo", "hi" or "all":
+    * step 0: the two diagonal chunk blocks (masked) and the high query chunk against the low
+      key chunk (wholly past);
+    * src < rank: both query chunks against the low key chunk (wholly past: one launch, the
+      two query chunks at their own positions);
+    * src > rank: the high query chunk against both key chunks (wholly past: one launch);
+    * blocks wholly in the future are skipped. Without the mask every step is one launch of
+      all queries against all keys.
+    Every rank attends 2*world chunk blocks (counting a diagonal one as half) in world + 2
+    launches under the mask."""
+    calls = []
     for t in range(world):
         src = (rank - t) % world
-        for qh in (0, 1):
-            for kh in (0, 1):
-                if not (causal and chunk(src, kh) > chunk(rank, qh)):
-                    out.append((t, src, qh, kh))
-    return out
+        if not causal:
+            calls.append((t, src, "all", "all", False))
+        elif t == 0:
+            calls += [(0, rank, "lo", "lo", True), (0, rank, "hi", "lo", False),
+                      (0, rank, "hi", "hi", True)]
+        elif src < rank:
+            calls.append((t, src, "all", "lo", False))
+        else:
+            calls.append((t, src, "hi", "all", False))
+    return calls
+
+
+def _zigzag_issue(partial_fn, calls, i, rank, world, c, q, k_cur, v_cur, acc_o, acc_l, out,
+                  rope_base):
+    """Launch call i of zigzag_calls on the views it names."""
+    t, src, qh, kh, masked = calls[i]
+    sl = {"lo": slice(0, c), "hi": slice(c, 2 * c), "all": slice(0, 2 * c)}
+
+    def pos(owner, half):
+        return (owner if half == "lo" else 2 * world - 1 - owner) * c
+
+    halves = ("lo", "hi") if qh == "all" else (qh,)
+    # the first call that writes a query half overwrites its accumulator rows
+    written = {h: any(calls[j][2] in (h, "all") for j in range(i)) for h in halves}
+    last = any(not any(calls[j][2] in (h, "all") for j in range(i + 1, len(calls)))
+               for h in halves)
+    q_pos0 = pos(rank, "hi" if qh == "hi" else "lo")
+    split, q_pos1 = (c, pos(rank, "hi")) if qh == "all" else (0, 0)
+    k_pos0 = pos(src, "hi" if kh == "hi" else "lo")
+    partial_fn(q[:, :, sl[qh]], k_cur[:, :, sl[kh]], v_cur[:, :, sl[kh]], acc_o[:, :, sl[qh]],
+               acc_l[:, :, sl[qh]], rope_base, q_pos0, k_pos0, causal=masked,
+               accumulate=all(written.values()), out=out[:, :, sl[qh]] if last else None,
+               q_split=split, q_pos1=q_pos1)
 
 
 def ring_attention(q, k, v, rope_base: float, causal: bool = True, group=None, out=None, *,
@@ -65,8 +99,8 @@ def ring_attention(q, k, v, rope_base: float, causal: bool = True, group=None, o
     rotated. Returns out [B, Hq, L, D] (bf16 through the library), this slice of the
     attention over the full sequence. Every rank of the group calls it with the same shapes.
     ``layout="zigzag"`` balances the causal work: the sequence is cut into 2*world chunks of
-    c tokens and rank r holds chunks r and 2*world-1-r, so q, k, v (and out, if given) are
-    pairs (first chunk, second chunk) of [B, H, c, D] tensors, and a pair is returned.
+    c tokens and rank r holds chunk r followed by chunk 2*world-1-r, so q, k, v (and out)
+    are [B, H, 2c, D] tensors in that order (see zigzag_calls).
     ``partial_fn`` / ``rotate_fn`` replace the library calls (same signatures as
     `rope_attn_fwd_partial` / `rope_attn_rotate`); the multi-process tests on CPU use them.
     """
@@ -123,33 +157,28 @@ def ring_attention(q, k, v, rope_base: float, causal: bool = True, group=None, o
 
 
 def _ring_zigzag(q, k, v, rope_base, causal, group, out, world, rank, partial_fn, rotate_fn):
-    """ring_attention with the zig-zag split (see zigzag_steps); q, k, v, out are pairs."""
-    if len(q) != 2 or len(k) != 2 or len(v) != 2:
-        raise ValueError("the zig-zag layout takes (first chunk, second chunk) pairs")
-    B, Hq, c, D = q[0].shape
-    for t in (q[1], k[0], k[1], v[0], v[1]):
-        if t.dim() != 4 or t.shape[0] != B or t.shape[2:] != (c, D):
-            raise ValueError("every chunk must be [B, H, c, D] with the same B, c and D")
-    if k[0].shape != k[1].shape or v[0].shape != k[0].shape or q[1].shape != q[0].shape:
-        raise ValueError("the two chunks of a pair must have the same shape")
+    """ring_attention with the zig-zag split: q, k, v, out are [B, H, 2c, D], chunk rank then
+    chunk 2*world-1-rank."""
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("q [B, Hq, 2c, D], k and v [B, Hkv, 2c, D]")
+    B, Hq, L, D = q.shape
+    if L % 2 or k.shape[0] != B or k.shape[2:] != (L, D):
+        raise ValueError("the zig-zag layout needs an even local length shared by q, k, v")
+    c = L // 2
 
     def peer(r):
         return r if group is None else dist.get_global_rank(group, r)
 
-    def pos(owner, half):
-        return (owner if half == 0 else 2 * world - 1 - owner) * c
-
-    own = [torch.empty_like(k[0]), torch.empty_like(k[1]), v[0], v[1]]
-    rotate_fn(k[0], rope_base, pos(rank, 0), out=own[0])
-    rotate_fn(k[1], rope_base, pos(rank, 1), out=own[1])
-    recv = [[torch.empty_like(x) for x in own] for _ in range(min(2, world - 1))]
-    acc = [(torch.empty((B, Hq, c, D), dtype=torch.float32, device=q[0].device),
-            torch.empty((B, Hq, c), dtype=torch.float32, device=q[0].device)) for _ in range(2)]
+    # own keys rotated at their two chunks' positions, values as given (read only)
+    own = (torch.empty_like(k), v)
+    rotate_fn(k[:, :, :c], rope_base, rank * c, out=own[0][:, :, :c])
+    rotate_fn(k[:, :, c:], rope_base, (2 * world - 1 - rank) * c, out=own[0][:, :, c:])
+    recv = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
+    acc_o = torch.empty((B, Hq, L, D), dtype=torch.float32, device=q.device)
+    acc_l = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     if out is None:
-        out = (torch.empty_like(q[0]), torch.empty_like(q[1]))
-    sched = zigzag_steps(rank, world, causal)
-    last = {qh: max(i for i, x in enumerate(sched) if x[2] == qh) for qh in (0, 1)}
-    first = {0: True, 1: True}
+        out = torch.empty_like(q)
+    calls = zigzag_calls(rank, world, causal)
     nxt, prv = peer((rank + 1) % world), peer((rank - 1) % world)
     i = 0
     for t in range(world):
@@ -157,16 +186,14 @@ def _ring_zigzag(q, k, v, rope_base, causal, group, out, world, rank, partial_fn
         reqs = []
         if t < world - 1:
             dst = recv[t % 2]
-            ops = [dist.P2POp(dist.isend, x, nxt, group) for x in cur]
-            ops += [dist.P2POp(dist.irecv, x, prv, group) for x in dst]
+            ops = [dist.P2POp(dist.isend, cur[0], nxt, group),
+                   dist.P2POp(dist.isend, cur[1], nxt, group),
+                   dist.P2POp(dist.irecv, dst[0], prv, group),
+                   dist.P2POp(dist.irecv, dst[1], prv, group)]
             reqs = dist.batch_isend_irecv(ops)
-        src = (rank - t) % world
-        while i < len(sched) and sched[i][0] == t:
-            _, _, qh, kh = sched[i]
-            partial_fn(q[qh], cur[kh], cur[2 + kh], acc[qh][0], acc[qh][1], rope_base,
-                       pos(rank, qh), pos(src, kh), causal=causal, accumulate=not first[qh],
-                       out=out[qh] if i == last[qh] else None)
-            first[qh] = False
+        while i < len(calls) and calls[i][0] == t:
+            _zigzag_issue(partial_fn, calls, i, rank, world, c, q, cur[0], cur[1], acc_o, acc_l,
+                          out, rope_base)
             i += 1
         for r in reqs:
             r.wait()
@@ -219,35 +246,41 @@ def ring_attention_local(q, k, v, rope_base: float, n_ranks: int, causal: bool =
 
 
 def _ring_zigzag_local(q, k, v, rope_base, n, causal, out, on_rank):
-    """ring_attention_local with the zig-zag split: chunk i of the sequence (c tokens at i*c)
-    is one contiguous tensor; rank r's blocks follow zigzag_steps."""
+    """ring_attention_local with the zig-zag split: each rank's [B, H, 2c, D] tensors are
+    assembled first (chunk r, chunk 2n-1-r; keys rotated at their positions), then every
+    rank's zigzag_calls run in turn on the other ranks' prepared keys and values."""
     B, Hq, S, D = q.shape
     if S % (2 * n):
         raise ValueError("the zig-zag split needs the sequence length a multiple of 2*n_ranks")
     c = S // (2 * n)
-    qs = [q[:, :, i * c:(i + 1) * c].contiguous() for i in range(2 * n)]
-    ks = [_lib.rope_attn_rotate(k[:, :, i * c:(i + 1) * c].contiguous(), rope_base, i * c)
-          for i in range(2 * n)]
-    vs = [v[:, :, i * c:(i + 1) * c].contiguous() for i in range(2 * n)]
-    outs = [torch.empty_like(qs[i]) for i in range(2 * n)]
-    acc = [(torch.empty((B, Hq, c, D), dtype=torch.float32, device=q.device),
-            torch.empty((B, Hq, c), dtype=torch.float32, device=q.device)) for _ in range(2)]
 
-    def chunk(owner, half):
-        return owner if half == 0 else 2 * n - 1 - owner
+    def rows(chunk):
+        return slice(chunk * c, (chunk + 1) * c)
 
+    mine = [(r, 2 * n - 1 - r) for r in range(n)]
+    qs = [torch.cat([q[:, :, rows(a)], q[:, :, rows(b)]], dim=2) for a, b in mine]
+    vs = [torch.cat([v[:, :, rows(a)], v[:, :, rows(b)]], dim=2) for a, b in mine]
+    ks = []
+    for a, b in mine:
+        kr = torch.empty((B, k.shape[1], 2 * c, D), dtype=k.dtype, device=k.device)
+        _lib.rope_attn_rotate(k[:, :, rows(a)], rope_base, a * c, out=kr[:, :, :c])
+        _lib.rope_attn_rotate(k[:, :, rows(b)], rope_base, b * c, out=kr[:, :, c:])
+        ks.append(kr)
+    outs = [torch.empty_like(x) for x in qs]
+    acc_o = torch.empty((B, Hq, 2 * c, D), dtype=torch.float32, device=q.device)
+    acc_l = torch.empty((B, Hq, 2 * c), dtype=torch.float32, device=q.device)
     for r in range(n):
         if on_rank:
             on_rank(r, "start")
-        sched = zigzag_steps(r, n, causal)
-        last = {qh: max(i for i, x in enumerate(sched) if x[2] == qh) for qh in (0, 1)}
-        first = {0: True, 1: True}
-        for i, (_, src, qh, kh) in enumerate(sched):
-            qi, ki = chunk(r, qh), chunk(src, kh)
-            _lib.rope_attn_fwd_partial(qs[qi], ks[ki], vs[ki], acc[qh][0], acc[qh][1], rope_base,
-                                       qi * c, ki * c, causal=causal, accumulate=not first[qh],
-                                       out=outs[qi] if i == last[qh] else None)
-            first[qh] = False
+        calls = zigzag_calls(r, n, causal)
+        for i, (_, src, _, _, _) in enumerate(calls):
+            _zigzag_issue(_lib.rope_attn_fwd_partial, calls, i, r, n, c, qs[r], ks[src], vs[src],
+                          acc_o, acc_l, outs[r], rope_base)
         if on_rank:
             on_rank(r, "end")
-    return torch.cat(outs, dim=2, out=out) if out is not None else torch.cat(outs, dim=2)
+    if out is None:
+        out = torch.empty_like(q)
+    for r, (a, b) in enumerate(mine):
+        out[:, :, rows(a)] = outs[r][:, :, :c]
+        out[:, :, rows(b)] = outs[r][:, :, c:]
+    return out
