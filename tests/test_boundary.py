@@ -257,3 +257,25 @@ def test_partial_noncausal_any_offsets_until_device(lib):
     # without the mask a block may sit anywhere; with no GPU the call fails at the device step
     st = partial(lib, qp=0, kp=500, causal=0)
     assert st != ra.RA_ERR_INVALID_ARG
+
+
+def test_view_rows_of_real_layouts():
+    import torch
+    # the binding's stride logic on CPU tensors of the layouts the entry points accept
+    from transformer_attention_04_b200._lib import view_rows
+    x = torch.empty(2, 3, 100, 64)
+    assert view_rows(tuple(x.shape), x.stride()) == 100                      # packed
+    v = x[:, :, 10:60]
+    assert view_rows(tuple(v.shape), v.stride()) == 100                      # slice along S
+    one = torch.empty(1, 5, 40, 64)[:, :, 8:24]
+    assert view_rows(tuple(one.shape), one.stride()) == 40                   # B = 1
+    single = torch.empty(3, 1, 40, 64)[:, :, :16]
+    assert view_rows(tuple(single.shape), single.stride()) == 40             # H = 1
+    lse = torch.empty(2, 3, 100)[:, :, 5:50]
+    assert view_rows(tuple(lse.shape), lse.stride()) == 100                  # 3-D accumulator
+    t = x.transpose(1, 2)                                                    # [B, S, H, D]
+    assert view_rows((2, 100, 3, 64), t.stride()) is None
+    cols = x[:, :, :, :32]                                                   # rows not packed
+    assert view_rows(tuple(cols.shape), cols.stride()) is None
+    heads = x[:, :2]                                                          # uneven batch step
+    assert view_rows(tuple(heads.shape), heads.stride()) is None

@@ -142,21 +142,38 @@ def rope_attn_prefill(q, k, v, rope_base: float, pos_offset: int = 0, causal: bo
     return out
 
 
+def view_rows(shape, stride):
+    """Rows between consecutive heads of a [B, H, S(, D)] layout whose rows are packed (a
+    slice along S of a longer tensor qualifies), or None if the layout is not of that form."""
+    B, H, S = shape[:3]
+    row = shape[3] if len(shape) == 4 else 1
+    if (len(shape) == 4 and stride[3] != 1 and row > 1) or (stride[2] != row and S > 1):
+        return None
+    if H > 1:
+        if stride[1] % row:
+            return None
+        rows = stride[1] // row
+    elif B > 1:
+        if stride[0] % row:
+            return None
+        rows = stride[0] // row
+    else:
+        rows = S
+    if rows < S or (B > 1 and stride[0] != H * rows * row):
+        return None
+    return rows
+
+
 def _head_rows(t, name, dtype, shape):
-    """Rows between consecutive heads of a [B, H, S(, D)] view whose rows are packed (a slice
-    along S of a longer tensor is allowed); checks dtype, device, shape and layout."""
+    """view_rows of a CUDA tensor, after checking its dtype, device and shape."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != dtype:
         raise ValueError(f"{name} must be a {dtype} CUDA tensor")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
-    B, H, S = shape[:3]
-    row = shape[3] if len(shape) == 4 else 1
-    st = t.stride()
-    if (len(shape) == 4 and st[3] != 1) or st[2] != row:
-        raise ValueError(f"{name}: rows must be packed along the last axis")
-    rows = st[1] // row if H > 1 else (st[0] // row if B > 1 else S)
-    if st[1] % row or rows < S or (B > 1 and st[0] != H * rows * row):
-        raise ValueError(f"{name}: heads must be evenly spaced slices of >= {S} rows")
+    rows = view_rows(tuple(shape), t.stride())
+    if rows is None:
+        raise ValueError(f"{name}: rows must be packed and heads evenly spaced slices of "
+                         f">= {shape[2]} rows")
     return rows
 
 
