@@ -738,3 +738,21 @@ def test_planted_zigzag_mistakes_are_caught(monkeypatch):
         (a, ((2 * n - 2 - r) * (S // (2 * n)), (2 * n - 1 - r) * (S // (2 * n))))
         for r, (a, _) in enumerate(orig(S, n))])
     assert not pin()
+
+
+def test_merge_is_associative_and_commutative():
+    # three partials over disjoint key ranges combine to the same result in any grouping/order
+    rng = np.random.default_rng(90)
+    q = rng.standard_normal((1, 2, 5, 8))
+    k_rot = ref.rope_rotate(rng.standard_normal((1, 1, 30, 8)), np.arange(30), 10000.0)
+    v = rng.standard_normal((1, 1, 30, 8))
+    parts = [oracle.rope_attn_fwd_partial(q, k_rot[:, :, a:b], v[:, :, a:b], 10000.0, 40, a, True)
+             for a, b in ((0, 7), (7, 19), (19, 30))]
+    m = oracle.merge_partials
+    left = m(*m(*parts[0], *parts[1]), *parts[2])
+    right = m(*parts[0], *m(*parts[1], *parts[2]))
+    swapped = m(*m(*parts[2], *parts[0]), *parts[1])
+    whole = oracle.rope_attn_fwd_partial(q, k_rot, v, 10000.0, 40, 0, True)
+    for o, lse in (left, right, swapped):
+        np.testing.assert_allclose(o, whole[0], atol=1e-13, rtol=0)
+        np.testing.assert_allclose(lse, whole[1], atol=1e-13, rtol=0)

@@ -195,3 +195,21 @@ def test_zigzag_calls_schedule():
                           for kc in range(2 * world) if kc <= qc)
             assert seen == want
             assert len(zigzag_calls(r, world, False)) == world
+
+
+def test_ring_drivers_reject_bad_arguments():
+    # argument errors are raised on the host before any library call (CPU tensors suffice)
+    sys.path.insert(0, ROOT)
+    from transformer_attention_04_b200.ring import ring_attention, ring_attention_local
+    q = torch.zeros(1, 4, 8, 16)
+    k = torch.zeros(1, 2, 8, 16)
+    with pytest.raises(ValueError):
+        ring_attention(q, k[:, :, :6], k, 1e4)                 # k shorter than q
+    with pytest.raises(ValueError):
+        ring_attention(q, k, k, 1e4, layout="striped")         # unknown layout
+    with pytest.raises(ValueError):
+        ring_attention(q[:, :, :7], k[:, :, :7], k[:, :, :7], 1e4, layout="zigzag")  # odd length
+    with pytest.raises(ValueError):
+        ring_attention_local(q, k, k, 1e4, 3)                  # 8 tokens over 3 ranks
+    with pytest.raises(ValueError):
+        ring_attention_local(q, k, k, 1e4, 3, layout="zigzag")  # 8 tokens over 6 chunks
