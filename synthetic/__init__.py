@@ -107,3 +107,23 @@ def make_inputs(w: Workload, seed: int = 0):
 def to_f64(t: torch.Tensor):
     """Exact widening of a bf16 tensor to a float64 numpy array."""
     return t.to(torch.float64).numpy()
+
+
+def plant_spikes(q: torch.Tensor, k: torch.Tensor, row_vals, key_pos, key_vals,
+                 key_pos0: int = 0) -> None:
+    """Overwrite the last two features of q and k in place (bf16 CPU tensors).
+
+    Query row i of every head gets (row_vals[i % len(row_vals)], 0); key row j of every head
+    gets (key_vals[n], 0) where key_pos0 + j == key_pos[n], and (0, 0) elsewhere. The other
+    features keep their N(0, 1) draw. Only values are written here: the caller chooses them.
+    """
+    D = q.shape[-1]
+    rv = torch.tensor([float(x) for x in row_vals], dtype=torch.float32)
+    idx = torch.arange(q.shape[2]) % len(row_vals)
+    q[..., D - 2] = rv[idx].to(q.dtype)
+    q[..., D - 1] = 0
+    k[..., D - 2:] = 0
+    for p, c in zip(key_pos, key_vals):
+        j = int(p) - key_pos0
+        if 0 <= j < k.shape[2]:
+            k[:, :, j, D - 2] = float(c)
