@@ -6,8 +6,11 @@ library instead of memory taken per call.
 
 The test calls the entry through the C ABI twice in a row, on different inputs (so a stale
 partial left by the first call would show in the second), and compares each result with the
-allocating rope_attn_decode within the parity tolerance of the other tests. It also checks
-that a request whose partials cannot fit the array is refused before anything is enqueued.
+allocating rope_attn_decode within the parity tolerance of the other tests, and once directly
+with the fp64 oracle. It also checks that the automatic split count is lowered until the
+partials fit (the result then equals the one-split allocating decode), and that a request
+whose partials cannot fit the array, even with one split, is refused before anything is
+enqueued.
 The file is named to be collected last.
 """
 import ctypes
@@ -15,8 +18,9 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 import transformer_attention_04_b200 as ra
-from parity_util import MAX_ABS, REL_RMS, errors
+from parity_util import MAX_ABS, REL_RMS, assert_parity, errors
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +59,53 @@ def test_noalloc_matches_decode_twice(shape):
         assert ra.rope_attn_get_device_status() == ra.RA_OK
         ma, rr = errors(out, ref.double().cpu().numpy())
         assert ma <= MAX_ABS and rr <= REL_RMS, (call, ma, rr)
+
+
+def _partials_bytes(B, Hq, D, splits):
+    rows = B * Hq * splits
+    return ((rows * D * 4 + 255) & ~255) + rows * 8
+
+
+def test_noalloc_matches_oracle():
+    B, Hq, Hkv, Sk, D, pos = 4, 16, 2, 3000, 128, 2999
+    q, kc, vc = _inputs(13, B, Hq, Hkv, Sk, D)
+    st, out = _noalloc(q, kc, vc, 500000.0, pos, 0)
+    assert st == ra.RA_OK, ra.lib().rope_attn_last_cuda_error()
+    torch.cuda.synchronize()
+    assert ra.rope_attn_get_device_status() == ra.RA_OK
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    assert_parity(out, oracle.rope_attn_decode(f(q), f(kc), f(vc), 500000.0, pos), "noalloc")
+
+
+def test_noalloc_lowers_the_automatic_split_count_to_fit():
+    # 21 x 800 query heads: the usual split count is 2 on a 148-SM B200, whose partials
+    # (16.7 MiB) do not fit the array; the entry lowers it to 1 split (8.3 MiB) and must
+    # then give what the allocating decode gives with one split
+    B, Hq, Hkv, Sk, D, pos = 21, 800, 10, 128, 128, 127
+    auto = ra.rope_attn_decode_auto_splits(B, Hq, Hkv, Sk, D, pos)
+    if auto < 2 or _partials_bytes(B, Hq, D, auto) <= SCRATCH_BYTES:
+        pytest.skip(f"the automatic split count here is {auto}; the shape is sized for 148 SMs")
+    assert _partials_bytes(B, Hq, D, 1) <= SCRATCH_BYTES
+    for seed in (14, 15):
+        q, kc, vc = _inputs(seed, B, Hq, Hkv, Sk, D)
+        ref = ra.rope_attn_decode(q, kc, vc, 500000.0, pos, n_splits=1)
+        st, out = _noalloc(q, kc, vc, 500000.0, pos, 0)
+        assert st == ra.RA_OK, ra.lib().rope_attn_last_cuda_error()
+        torch.cuda.synchronize()
+        assert ra.rope_attn_get_device_status() == ra.RA_OK
+        ma, rr = errors(out, ref.double().cpu().numpy())
+        assert ma <= MAX_ABS and rr <= REL_RMS, (seed, ma, rr)
+
+
+def test_noalloc_refuses_when_one_split_does_not_fit():
+    # 128 x 256 heads need 16.25 MiB of partials even with a single split
+    B, Hq, Hkv, Sk, D = 128, 256, 8, 64, 128
+    assert _partials_bytes(B, Hq, D, 1) > SCRATCH_BYTES
+    q = torch.zeros(B, Hq, 1, D, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(B, Hkv, Sk, D, dtype=torch.bfloat16, device="cuda")
+    st, _ = _noalloc(q, kc, kc.clone(), 500000.0, Sk - 1, 0)
+    assert st == ra.RA_ERR_UNSUPPORTED
+    assert b"scratch" in ra.lib().rope_attn_last_cuda_error()
 
 
 def test_noalloc_rejects_partials_beyond_scratch():
