@@ -209,6 +209,10 @@ def test_ring_drivers_reject_bad_arguments():
         ring_attention(q, k, k, 1e4, layout="striped")         # unknown layout
     with pytest.raises(ValueError):
         ring_attention(q[:, :, :7], k[:, :, :7], k[:, :, :7], 1e4, layout="zigzag")  # odd length
+    with pytest.raises(ValueError, match="contiguous"):
+        ring_attention(q, k, torch.zeros(1, 2, 12, 16)[:, :, :8], 1e4)  # v a slice of a longer v
+    with pytest.raises(ValueError, match="contiguous"):
+        ring_attention(q, torch.zeros(1, 2, 12, 16)[:, :, 4:], k, 1e4, layout="zigzag")
     with pytest.raises(ValueError):
         ring_attention_local(q, k, k, 1e4, 3)                  # 8 tokens over 3 ranks
     with pytest.raises(ValueError):

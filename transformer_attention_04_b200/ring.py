@@ -78,8 +78,13 @@ def _zigzag_issue(partial_fn, calls, i, rank, world, c, q, k_cur, v_cur, acc_o, 
         return (owner if half == "lo" else 2 * world - 1 - owner) * c
 
     halves = ("lo", "hi") if qh == "all" else (qh,)
-    # the first call that writes a query half overwrites its accumulator rows
+    # the first call that writes a query half overwrites its accumulator rows; one call can
+    # only overwrite or merge all the rows it covers, so its halves must agree
     written = {h: any(calls[j][2] in (h, "all") for j in range(i)) for h in halves}
+    if len(set(written.values())) != 1:
+        raise RuntimeError(f"zig-zag call {i} covers a written and an unwritten query half")
+    # bf16 rows are written by a half's final call; an "all" call that is final for the low
+    # half also writes the high half's rows, which that half's final call overwrites later
     last = any(not any(calls[j][2] in (h, "all") for j in range(i + 1, len(calls)))
                for h in halves)
     q_pos0 = pos(rank, "hi" if qh == "hi" else "lo")
@@ -106,6 +111,11 @@ def ring_attention(q, k, v, rope_base: float, causal: bool = True, group=None, o
     """
     partial_fn = partial_fn or _lib.rope_attn_fwd_partial
     rotate_fn = rotate_fn or _lib.rope_attn_rotate
+    # k and v are sent whole to the next rank, and the received blocks must have v's layout
+    for name, t in (("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [B, Hkv, L, D] tensor: the ring "
+                             f"sends it whole to the next rank")
     distributed = dist.is_available() and dist.is_initialized()
     world = dist.get_world_size(group) if distributed else 1
     rank = dist.get_rank(group) if distributed else 0
