@@ -332,6 +332,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (lane == 0) mbar_arrive(empty(st));
   }
 
+  // every tile is consumed: the combine kernel may be scheduled now (its CTAs wait in
+  // grid_dep_wait until this grid has completed and written its partials)
+  grid_dep_launch();
   // reduce the per-lane sums over the 8 lanes that share a head column
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
@@ -378,10 +381,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 }
 
-// the merge of the splits: out[b, h, 0, :] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
+// the merge of the splits: out[b, h, 0, :] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+// Launched right behind the split kernel with a programmatic dependency, so its launch
+// overlaps the split kernel's last wave; it reads the partials only after grid_dep_wait.
 __global__ void decode_combine_kernel(const float* __restrict__ part_o,
                                       const float2* __restrict__ part_ml,
                                       __nv_bfloat16* __restrict__ out, int n_splits, int D) {
+  grid_dep_wait();
   const long long bh = blockIdx.x;
   const float2* ml = part_ml + bh * n_splits;
   float M = -INFINITY;

@@ -279,16 +279,17 @@ struct PrefillArgs {
   int window;
 };
 
-// One launch of the attention kernel: one CTA per work unit (query tile, batch, KV group,
-// query-head pair); blockIdx order is longest causal extent first.
+// One launch of the persistent attention kernel: one CTA per SM (fewer when there are fewer
+// work units), each walking its units (query tile, batch, KV group, query-head pair) of the
+// longest-first order in snake order.
 ra_status launch_attn(const ra::FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                      const CUtensorMap& tv, int D, long long n_units, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>(n_units));
+                      const CUtensorMap& tv, int D, int num_sms, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(std::min<long long>(p.n_units, num_sms)));
   const int pi = prof_start(0, s);
   if (D == 64)
-    ra::attn_fwd_sm100_kernel<64><<<grid, 384, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
+    ra::attn_fwd_sm100_kernel<64><<<grid, ra::kFwdThreads, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
   else
-    ra::attn_fwd_sm100_kernel<128><<<grid, 384, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
+    ra::attn_fwd_sm100_kernel<128><<<grid, ra::kFwdThreads, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
   prof_stop(0, pi, s);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "attn_fwd launch");
@@ -384,16 +385,19 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.n_slots = n_slots;
     p.ppg = G / n_slots;
     p.n_qtiles = n_qtiles;
+    p.n_units = static_cast<int>(n_units);
     p.causal = a.causal ? 1 : 0;
     p.off = static_cast<int>(T) - Sq;  // bottom-right alignment of the queries on the keys
     p.window = a.window;
     p.q_tab_off = (Sk - Sq) - tab_lo;
+    p.q_split = Sq;
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+    p.rope_base = a.rope_base;
     p.o_acc = nullptr;
     p.lse_acc = nullptr;
     p.accumulate = 0;
     p.acc_rows = Sq;
-    rs = launch_attn(p, tq, tk, tv, D, n_units, s);
+    rs = launch_attn(p, tq, tk, tv, D, ds->num_sms, s);
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
   if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
@@ -504,16 +508,19 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
     p.n_slots = n_slots;
     p.ppg = G / n_slots;
     p.n_qtiles = n_qtiles;
+    p.n_units = static_cast<int>(n_units);
     p.causal = a.causal ? 1 : 0;
     p.off = a.q_pos0 - a.k_pos0;  // query row i at q_pos0 + i, key j at k_pos0 + j
     p.window = 0;
     p.q_tab_off = 0;
+    p.q_split = n0;  // table row n0 starts the second segment's positions (Sq: none)
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
+    p.rope_base = a.rope_base;
     p.o_acc = a.o_acc;
     p.lse_acc = a.lse_acc;
     p.accumulate = a.accumulate ? 1 : 0;
     p.acc_rows = acc_rows;
-    rs = launch_attn(p, tq, tk, tv, D, n_units, s);
+    rs = launch_attn(p, tq, tk, tv, D, ds->num_sms, s);
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
   if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
@@ -684,9 +691,24 @@ ra_status decode_impl(const DecodeArgs& a, cudaStream_t s) {
   else
     ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
   prof_stop(1, pi, s);
-  ra::decode_combine_kernel<<<static_cast<unsigned>(B * Hq), D, 0, s>>>(
-      p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(a.out), splits, D);
   cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    // the combine may launch while the split kernel's last wave runs (it waits on the
+    // device for the split grid to complete before reading the partials)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(B * Hq));
+    cfg.blockDim = dim3(static_cast<unsigned>(D));
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, ra::decode_combine_kernel, static_cast<const float*>(p.part_o),
+                           static_cast<const float2*>(p.part_ml),
+                           static_cast<__nv_bfloat16*>(a.out), splits, D);
+  }
   if (e != cudaSuccess) rs = cuda_fail(e, "decode launch");
   if (!a.noalloc) {
     cudaError_t ef = cudaFreeAsync(ws, s);
@@ -920,13 +942,5 @@ ra_status rope_attn_decode_paged(const void* q, const void* k_new, const void* v
   return decode_impl(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
-#ifdef RA_TRACE
-// Profiling builds only: copy the phase stamps of the last prefill launch to the host.
-RA_API int rope_attn_trace_read(void* host, size_t bytes) {
-  if (bytes < sizeof(ra::g_trace)) return RA_ERR_INVALID_ARG;
-  return cudaMemcpyFromSymbol(host, ra::g_trace, sizeof(ra::g_trace)) == cudaSuccess ? RA_OK
-                                                                                      : RA_ERR_CUDA;
-}
-#endif
 
 }  // extern "C"
