@@ -62,8 +62,9 @@ struct FwdParams {
   int causal;
   int off;              // query row i sits at key index i + off (causal: key j allowed iff j <= i + off)
   int window;           // 0 = none; else key j is allowed to query row i iff j > i + off - window
-  int q_tab_off;        // table row of query row 0 (table rows are consecutive positions...)
-  int q_split;          // (...except at this query row, where a second segment starts; Sq if none)
+  int q_tab_off;        // query row i < q_split reads table row q_tab_off + i
+  int q_split;          // first row of a second segment of positions (Sq if none)...
+  int q_tab_off2;       // ...whose row i reads table row q_tab_off2 + i
   float scale_log2;     // log2(e) / sqrt(D)
   float rope_base;
   // partial (ring) mode when o_acc is set: O / l in fp32 [B, Hq, Sq, D] and the row's natural
@@ -142,8 +143,7 @@ __device__ __forceinline__ int unit_of(const FwdParams& p, int k) {
 
 // P = 2^(s * sl2 - m) for one 128-column row of S held in registers; writes the bf16 P
 // over the first 64 TMEM columns at tS and returns the row sum of the fp32 values.
-// Pairs go through one packed FMA; kEmu of every 4 pairs use the FMA-pipe exponential.
-template <int kEmu>
+// Pairs go through one packed FMA; the exponentials run on the MUFU.
 __device__ __forceinline__ float softmax_p_store(const uint32_t* sr, float sl2, float m,
                                                  uint32_t tS) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -157,17 +157,10 @@ __device__ __forceinline__ float softmax_p_store(const uint32_t* sr, float sl2, 
       const int c = h * 64 + 2 * c2;
       const uint64_t x2 =
           f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
-      uint64_t p2;
-      if ((c2 & 3) < kEmu) {
-        p2 = exp2_poly_x2(x2);
-      } else {
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
-        p2 = f2_pack(ex2(x0), ex2(x1));
-      }
-      acc2[c2 & 1] = f2_add(acc2[c2 & 1], p2);
-      float p0, p1;
-      f2_unpack(p2, p0, p1);
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      const float p0 = ex2(x0), p1 = ex2(x1);
+      acc2[c2 & 1] = f2_add(acc2[c2 & 1], f2_pack(p0, p1));
       pk[c2] = pack_bf16(p0, p1);
     }
     tmem_st32(tS + 32 * h, pk);
@@ -178,55 +171,7 @@ __device__ __forceinline__ float softmax_p_store(const uint32_t* sr, float sl2, 
   return a0 + a1;
 }
 
-// Same as softmax_p_store, and also returns the max of the 128 raw scores in `mt` (four
-// independent 3-input max chains interleaved with the exponentials, off the critical path).
-template <int kEmu>
-__device__ __forceinline__ float softmax_p_store_max(const uint32_t* sr, float sl2, float m,
-                                                     uint32_t tS, float& mt) {
-  const uint64_t sl2x2 = f2_pack(sl2, sl2);
-  const uint64_t negm2 = f2_pack(-m, -m);
-  uint64_t acc2[2] = {0, 0};
-  float mx[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) mx[k] = -INFINITY;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int c2 = 0; c2 < 32; ++c2) {
-      const int c = h * 64 + 2 * c2;
-      const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
-      mx[c2 & 3] = max3f(mx[c2 & 3], s0, s1);
-      const uint64_t x2 = f2_fma(f2_pack(s0, s1), sl2x2, negm2);
-      uint64_t p2;
-      if ((c2 & 3) < kEmu) {
-        p2 = exp2_poly_x2(x2);
-      } else {
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
-        p2 = f2_pack(ex2(x0), ex2(x1));
-      }
-      acc2[c2 & 1] = f2_add(acc2[c2 & 1], p2);
-      float p0, p1;
-      f2_unpack(p2, p0, p1);
-      pk[c2] = pack_bf16(p0, p1);
-    }
-    tmem_st32(tS + 32 * h, pk);
-  }
-  mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-  const uint64_t a = f2_add(acc2[0], acc2[1]);
-  float a0, a1;
-  f2_unpack(a, a0, a1);
-  return a0 + a1;
-}
-
-#ifndef RA_EMU_PAIRS
-#define RA_EMU_PAIRS 0
-#endif
-
-// kEmuPairs: of every 4 column pairs of an unmasked tile, how many take the FMA-pipe
-// exponential (0 = all on the MUFU).
-template <int D, int kEmuPairs = RA_EMU_PAIRS>
+template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -278,6 +223,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // launched behind the key rotation with a programmatic dependency: the set-up above overlaps
+  // its tail, the rotated keys and the table are read only after it has completed
+  grid_dep_wait();
 
   // Register split: launched at 168 per thread (384 x 168 = 64512); the control
   // warpgroup gives back to 80, the two softmax warpgroups take 208
@@ -342,93 +290,94 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
+    // One thread issues every MMA, in the order PV0(t) S0(t+1) PV1(t) S1(t+1) per tile t
+    // (S(t+1) being the S of the unit's next tile, or the next unit's first). The single
+    // order makes the two slots alternate: one slot's softmax runs while the other slot's
+    // MMAs execute. Each tcgen05.mma holds the issuing thread for about its duration and
+    // each barrier wait or commit costs it a few hundred cycles, so the thread keeps the
+    // code between MMAs short and waits for the ring tiles while it would wait for P anyway.
     if (lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc_bf16(128, 128, 0, 0);  // Q, K both K-major
       constexpr uint32_t kIdescO = umma_idesc_bf16(128, D, 0, 1);    // V is MN-major
-      // shared-memory descriptors are formed from 32-bit addresses at issue time (their
-      // upper half is a constant), which keeps the issuing thread's live state small
+      constexpr uint32_t kHi = umma_desc_hi_sw128(1024);
+      // low descriptor words of Q tile 0 and of ring slot 0 (as the B operand of S, and as V
+      // for PV); other tiles and slots add a multiple of TILE >> 4
+      const uint32_t q_lo0 = umma_desc_lo(sQ, 16);
+      const uint32_t k_lo0 = umma_desc_lo(sRing, 16);
+      const uint32_t v_lo0 = umma_desc_lo(sRing, C::BLK);
       auto issue_s = [&](int qtile, int s, int sl) {  // qtile = Q buffer * 2 + slot
         const uint32_t d_t = tmem + C::col_s(s);
-        const uint32_t a = sQ + qtile * C::TILE, bq = sRing + sl * C::TILE;
+        const uint32_t qlo = q_lo0 + static_cast<uint32_t>(qtile * (C::TILE >> 4));
+        const uint32_t klo = k_lo0 + static_cast<uint32_t>(sl * (C::TILE >> 4));
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t o = (k >> 2) * C::BLK + (k & 3) * 32;
-          umma_ss(d_t, umma_smem_desc(a + o, 16, 1024, kLayoutSW128),
-                  umma_smem_desc(bq + o, 16, 1024, kLayoutSW128), kIdescS, k > 0 ? 1u : 0u);
+          constexpr uint32_t kBlk = C::BLK >> 4;
+          const uint32_t o = static_cast<uint32_t>((k >> 2) * kBlk + (k & 3) * 2);
+          umma_ss(d_t, umma_desc(qlo + o, kHi), umma_desc(klo + o, kHi), kIdescS, k > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int s, int sl, bool acc) {
         const uint32_t d_t = tmem + C::col_o(s);
         const uint32_t a_t = tmem + C::col_s(s);
-        const uint32_t bv = sRing + sl * C::TILE;
+        const uint32_t vlo = v_lo0 + static_cast<uint32_t>(sl * (C::TILE >> 4));
 #pragma unroll
         for (int k = 0; k < 8; ++k)  // 128 keys, 16 per MMA
-          umma_ts(d_t, a_t + 8 * k, umma_smem_desc(bv + k * 2048, C::BLK, 1024, kLayoutSW128),
+          umma_ts(d_t, a_t + 8 * k, umma_desc(vlo + static_cast<uint32_t>(k * (2048 >> 4)), kHi),
                   kIdescO, (acc || k > 0) ? 1u : 0u);
       };
       // global tile t: K item 2t, V item 2t + 1
       auto slot = [](int item) { return item % C::NSLOT; };
       auto par = [](int item) { return static_cast<uint32_t>((item / C::NSLOT) & 1); };
-
-      // S of the first tile of unit k (tile counter t)
-      auto first_s = [&](int k, int t, int n_it) -> bool {
-        const int qb = k & 1;
-        if (!mbar_wait(bar(C::B_QREADY + qb), (k >> 1) & 1, lim, abort_flag, p.status) ||
-            !mbar_wait(bar(C::B_FULL + slot(2 * t)), par(2 * t), lim, abort_flag, p.status))
-          return false;
-        issue_s(qb * 2 + 0, 0, slot(2 * t));
-        umma_commit(bar(C::B_SFULL + 0));
-        if (ns == 2) {
-          issue_s(qb * 2 + 1, 1, slot(2 * t));
-          umma_commit(bar(C::B_SFULL + 1));
-        }
-        if (n_it == 1) umma_commit(bar(C::B_QEMPTY + qb));
-        umma_commit(bar(C::B_EMPTY + slot(2 * t)));
-        return true;
+      auto wait = [&](int b, uint32_t parity) {
+        return mbar_wait(bar(b), parity, lim, abort_flag, p.status);
       };
 
+      bool ok = false;
+      int n_it = 0;
+      const int u0 = unit_of(p, 0);
+      if (u0 >= 0) {
+        n_it = unit_at(p, u0).n_it;
+        // S of unit 0's first tile
+        ok = wait(C::B_QREADY + 0, 0) && wait(C::B_FULL + slot(0), par(0));
+        if (ok) {
+          issue_s(0, 0, slot(0));
+          umma_commit(bar(C::B_SFULL + 0));
+          if (ns == 2) {
+            issue_s(1, 1, slot(0));
+            umma_commit(bar(C::B_SFULL + 1));
+          }
+          if (n_it == 1) umma_commit(bar(C::B_QEMPTY + 0));
+          umma_commit(bar(C::B_EMPTY + slot(0)));
+        }
+      }
       int t = 0;
-      bool ok = unit_of(p, 0) >= 0;
-      Unit w = ok ? unit_at(p, unit_of(p, 0)) : Unit{};
-      ok = ok && first_s(0, 0, w.n_it);
       for (int k = 0; ok; ++k) {
-        const int n_it = w.n_it;
-        Unit wn = w;
+        const int nu = unit_of(p, k + 1);
+        const int n_next = nu >= 0 ? unit_at(p, nu).n_it : 0;
         for (int jj = 0; ok && jj < n_it; ++jj, ++t) {
           const bool last = jj + 1 == n_it;
-          // the tile after this one: in this unit, or the first of the next unit
-          const int nu = last ? unit_of(p, k + 1) : -1;
-          const bool has_next = !last || nu >= 0;
-          if (last && nu >= 0) wn = unit_at(p, nu);
-          const int kn = last ? k + 1 : k;   // unit of the next tile
-          const int jn = last ? 0 : jj + 1;  // its index in that unit
-          const int qbn = kn & 1;
+          const bool has_next = !last || n_next > 0;
+          const int qbn = last ? (k + 1) & 1 : k & 1;                  // Q buffer of the next tile
+          const bool next_last = last ? n_next == 1 : jj + 2 == n_it;  // next tile ends its unit
+          // the ring tiles (normally landed long ago) and the next unit's Q first, then P0
+          ok = wait(C::B_FULL + slot(2 * t + 1), par(2 * t + 1)) &&
+               (!has_next || ((!last || wait(C::B_QREADY + qbn, ((k + 1) >> 1) & 1)) &&
+                              wait(C::B_FULL + slot(2 * t + 2), par(2 * t + 2)))) &&
+               wait(C::B_PFULL + 0, t & 1);
+          if (!ok) break;
           // ---- slot 0: PV0(t), then S0(t + 1)
           // (P_s of a unit's first tile comes after the softmax group has read the previous
           // unit's O_s, so PV_s may overwrite it)
-          if (!mbar_wait(bar(C::B_PFULL + 0), t & 1, lim, abort_flag, p.status) ||
-              !mbar_wait(bar(C::B_FULL + slot(2 * t + 1)), par(2 * t + 1), lim, abort_flag,
-                         p.status)) {
-            ok = false;
-            break;
-          }
           tc_fence_after();
           issue_pv(0, slot(2 * t + 1), jj > 0);
           if (last) umma_commit(bar(C::B_OFULL + 0));
           if (has_next) {
-            if ((jn == 0 && !mbar_wait(bar(C::B_QREADY + qbn), (kn >> 1) & 1, lim, abort_flag,
-                                       p.status)) ||
-                !mbar_wait(bar(C::B_FULL + slot(2 * t + 2)), par(2 * t + 2), lim, abort_flag,
-                           p.status)) {
-              ok = false;
-              break;
-            }
             issue_s(qbn * 2 + 0, 0, slot(2 * t + 2));
             umma_commit(bar(C::B_SFULL + 0));
           }
           // ---- slot 1: PV1(t), then S1(t + 1)
           if (ns == 2) {
-            if (!mbar_wait(bar(C::B_PFULL + 1), t & 1, lim, abort_flag, p.status)) {
+            if (!wait(C::B_PFULL + 1, t & 1)) {
               ok = false;
               break;
             }
@@ -442,12 +391,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           umma_commit(bar(C::B_EMPTY + slot(2 * t + 1)));
           if (has_next) {
-            if (jn + 1 == wn.n_it) umma_commit(bar(C::B_QEMPTY + qbn));  // its unit's last S
+            if (next_last) umma_commit(bar(C::B_QEMPTY + qbn));  // that unit's last S
             umma_commit(bar(C::B_EMPTY + slot(2 * t + 2)));
           }
-          if (last && nu < 0) ok = false;  // no more units: leave both loops
         }
-        w = wn;
+        if (!ok || n_next == 0) break;
+        n_it = n_next;
       }
       // every MMA issued above must finish before TMEM is released
       umma_commit(bar(C::B_DRAIN));
@@ -492,8 +441,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int row = rb0 + rr, qr = w.q0 + row;
         if (qr >= p.Sq) break;
         if (rr == 0 || qr == p.q_split) {
+          const int trow = (qr < p.q_split ? p.q_tab_off : p.q_tab_off2) + qr;
           const float4* t4 = reinterpret_cast<const float4*>(
-              p.tab + static_cast<long long>(p.q_tab_off + qr) * (D / 2) + ck * 4);
+              p.tab + static_cast<long long>(trow) * (D / 2) + ck * 4);
           const float4 a = __ldg(t4), b2 = __ldg(t4 + 1);
           cs[0] = make_float2(a.x, a.y);
           cs[1] = make_float2(a.z, a.w);
@@ -564,18 +514,20 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (c > lim_k || c < lo_k) sr[c] = 0xff800000u;  // -inf
         }
         // online softmax with a lazily updated reference max m. Once a row has a
-        // reference, P is computed speculatively with it while the tile max is gathered
-        // on the side; only if some row's max grew by more than 8 (log2 units) does the warp
-        // redo the tile exactly (rescale O, P with the new reference). Either way every row
-        // ends with the same values as the plain max-first order.
+        // reference, P is computed speculatively with it; every p is then at most 2^8 unless
+        // the tile's row sum exceeds 2^8. Only then does the warp take the tile's max and, if
+        // some row's max grew by more than 8 (log2 units), redo the tile exactly (rescale O,
+        // P with the new reference). Either way every row ends with the same values as the
+        // plain max-first order.
         float rs = 0.f;
         bool done = false;
         float mt = -INFINITY;
         if (!__any_sync(0xffffffffu, m == -INFINITY)) {
-          rs = need_mask ? softmax_p_store_max<0>(sr, sl2, m, tS, mt)
-                         : softmax_p_store_max<kEmuPairs>(sr, sl2, m, tS, mt);
-          done = !__any_sync(0xffffffffu, fmaxf(m, mt * sl2) > m + 8.0f);
-        } else {
+          rs = softmax_p_store(sr, sl2, m, tS);
+          // every p <= 2^8 unless the tile's row sum exceeds 2^8 (or is inf / NaN)
+          done = !__any_sync(0xffffffffu, !(rs <= 256.0f));
+        }
+        if (!done) {
           // tile max of the raw scores: eight independent 3-input max chains, then a tree
           float mx[8];
 #pragma unroll
@@ -614,8 +566,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           // p = 2^(s * log2(e)/sqrt(D) - m) -> bf16 P over the S columns; a row that has seen
           // no allowed key yet (only under a window) keeps m = -inf and gets P = 0
           const float m_use = (m == -INFINITY) ? 0.f : m;
-          rs = need_mask ? softmax_p_store<0>(sr, sl2, m_use, tS)
-                         : softmax_p_store<kEmuPairs>(sr, sl2, m_use, tS);
+          rs = softmax_p_store(sr, sl2, m_use, tS);
         }
         l += rs;
         tmem_wait_st();

@@ -41,6 +41,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase of parity `parity` (the thread is never suspended).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Spinning form of mbar_wait for a thread on the critical path: polls with test_wait, so
+// it sees the phase complete within a few cycles instead of after a suspension. Same limit,
+// status and abort rules as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, long long limit,
+                                               volatile int* abort_flag, unsigned int* status) {
+  for (long long i = 0; i < limit; ++i) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+  }
+  if (limit > 0 && mbar_test_wait(bar, parity)) return true;
+  *abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
 // Wait for the phase of parity `parity` of barrier `bar` to complete, polling at
 // most `limit` times. On running out it records kStatusTimeout in the sticky
 // device status word, raises the CTA's abort flag and returns false; a raised
@@ -54,6 +82,51 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
   }
   // limit 0 gives up without looking (a wait that nothing can satisfy, for tests)
   if (limit > 0 && mbar_try_wait(bar, parity)) return true;
+  *abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
+// Two phases polled together: both queries are in flight at once, so a pair of barriers
+// that have already completed costs one round trip instead of two.
+__device__ __forceinline__ bool mbar_wait2(uint32_t bar1, uint32_t parity1, uint32_t bar2,
+                                           uint32_t parity2, long long limit,
+                                           volatile int* abort_flag, unsigned int* status) {
+  bool d1 = false, d2 = false;
+  for (long long i = 0; i < limit; ++i) {
+    d1 = d1 || mbar_try_wait(bar1, parity1);
+    d2 = d2 || mbar_try_wait(bar2, parity2);
+    if (d1 && d2) return true;
+    if (*abort_flag) return false;
+  }
+  if (limit > 0 && (d1 || mbar_try_wait(bar1, parity1)) && (d2 || mbar_try_wait(bar2, parity2)))
+    return true;
+  *abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
+// Shared-memory event counters: a cheaper signal than an mbarrier between threads of one CTA
+// (a poll is one load). The producer side adds with release semantics, the consumer loads
+// with acquire semantics; together with tcgen05.fence::before/after_thread_sync on either
+// side this orders tcgen05 operations across the two threads.
+__device__ __forceinline__ void smem_add_release(uint32_t addr, uint32_t v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t smem_ld_acquire(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+// Wait until the counter at `addr` reaches `target` (counters only grow), with the same
+// limit, status and abort rules as mbar_wait.
+__device__ __forceinline__ bool smem_wait_count(uint32_t addr, uint32_t target, long long limit,
+                                                volatile int* abort_flag, unsigned int* status) {
+  for (long long i = 0; i < limit; ++i) {
+    if (static_cast<int>(smem_ld_acquire(addr) - target) >= 0) return true;
+    if (*abort_flag) return false;
+  }
+  if (limit > 0 && static_cast<int>(smem_ld_acquire(addr) - target) >= 0) return true;
   *abort_flag = 1;
   atomicOr(status, kStatusTimeout);
   return false;
@@ -74,6 +147,22 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, lo
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
   }
   const bool ok = limit > 0 && __all_sync(0xffffffffu, mbar_try_wait(bar, parity));
+  if (!ok && (threadIdx.x & 31) == 0) {
+    *abort_flag = 1;
+    atomicOr(status, kStatusTimeout);
+  }
+  __syncwarp();
+  return ok;
+}
+
+// Warp-collective spinning wait (test_wait polls; see mbar_wait_spin).
+__device__ __forceinline__ bool mbar_wait_warp_spin(uint32_t bar, uint32_t parity, long long limit,
+                                                    volatile int* abort_flag, unsigned int* status) {
+  for (long long i = 0; i < limit; ++i) {
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
+  }
+  const bool ok = limit > 0 && __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
   if (!ok && (threadIdx.x & 31) == 0) {
     *abort_flag = 1;
     atomicOr(status, kStatusTimeout);
@@ -258,6 +347,20 @@ __device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr, uint32_t lbo_
 }
 constexpr uint32_t kLayoutSW128 = 2;  // 128-byte swizzle
 
+// The same descriptor split in two 32-bit words: the low word holds the start address and
+// the leading byte offset, the high word the stride byte offset, the version bit and the
+// 128-byte swizzle. A k-step inside a tile is then a 32-bit add on the low word (shared
+// memory addresses stay below 256 KB, so the 14-bit address field cannot carry over).
+__device__ __forceinline__ uint32_t umma_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t umma_desc_hi_sw128(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (kLayoutSW128 << 29);
+}
+__device__ __forceinline__ uint64_t umma_desc(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 // a_mn / b_mn: 1 when that operand is MN-major in shared memory.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, int b_mn) {
@@ -338,31 +441,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for two arguments on the FMA pipe (keeps the MUFU free for the other exponentials).
-// x = n + f with n = round(x) taken from the low bits of x + 1.5*2^23 and f in [-1/2, 1/2];
-// 2^f is the cubic fitted by csrc/exp2_poly_fit.py (minimax relative error 7.5e-5), and 2^n
-// is added to the exponent field. Arguments are clamped at -120 (2^-120 is negligible next
-// to a softmax row sum >= 1); callers keep -inf (masked) entries away from this routine.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
-  const uint64_t kMagic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t kNegMagic = f2_pack(-12582912.0f, -12582912.0f);
-  const uint64_t kNegOne = f2_pack(-1.0f, -1.0f);
-  const uint64_t t = f2_add(xc, kMagic);
-  const uint64_t n = f2_add(t, kNegMagic);
-  const uint64_t f = f2_fma(n, kNegOne, xc);
-  uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
-                      f2_pack(2.426111251e-01f, 2.426111251e-01f));
-  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
-  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
-                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
-}
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
 }  // namespace ra

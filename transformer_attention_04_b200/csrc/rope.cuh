@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* __restric
                                                           long long nrows_total, int S, int D,
                                                           long long pos0, int tab_off,
                                                           float base, int x_rows, int y_rows) {
+  // the attention kernel launched next may start its set-up now (it waits for this grid)
+  grid_dep_launch();
   // x_rows / y_rows: rows between consecutive heads of x and y (S when packed)
   const int cpr = D / 8;  // 16-byte chunks per row
   const long long n = nrows_total * cpr;
@@ -102,6 +104,7 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restric
                                                           const float2* __restrict__ tab,
                                                           long long bh_count, int S, int S_cache,
                                                           int pos0, int D, int tab_off) {
+  grid_dep_launch();  // as in rope_rotate_kernel
   const int cpr = D / 8;
   const long long n = bh_count * S * cpr;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;

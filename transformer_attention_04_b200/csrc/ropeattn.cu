@@ -258,6 +258,75 @@ size_t decode_partials_bytes(int B, int Hq, int D, int splits) {
   return po + rows * sizeof(float2);
 }
 
+// ------------------------------------------------------------------ RoPE table cache
+// (cos, sin) of absolute positions 0 .. rows-1 for one (device, base, D), built once and kept
+// for the life of the process, so that a prefill or ring block does not rebuild its table.
+// A table grows to the next power of two of the positions a call needs; a grown table
+// replaces the old one, which stays allocated (calls already enqueued may read it).
+struct RopeTable {
+  int dev;
+  uint32_t base_bits;
+  int D;
+  long long rows;
+  float2* ptr;
+};
+constexpr size_t kTabCacheMaxBytes = static_cast<size_t>(64) << 20;
+std::mutex g_tab_mu;
+std::vector<RopeTable> g_tabs;
+std::vector<float2*> g_tabs_retired;
+
+// Sets *out to a table covering positions 0 .. rows_needed-1, or to null when the call must
+// build its own (too many positions, or the stream is being captured into a graph, where the
+// synchronous set-up of a new table is not possible).
+ra_status cached_table(const DeviceState* ds, float base, int D, long long rows_needed,
+                       cudaStream_t s, const float2** out) {
+  *out = nullptr;
+  const size_t row_bytes = static_cast<size_t>(D / 2) * sizeof(float2);
+  if (rows_needed <= 0 || static_cast<size_t>(rows_needed) * row_bytes > kTabCacheMaxBytes)
+    return RA_OK;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  uint32_t bits = 0;
+  std::memcpy(&bits, &base, sizeof(bits));
+  std::lock_guard<std::mutex> lock(g_tab_mu);
+  RopeTable* hit = nullptr;
+  for (RopeTable& t : g_tabs)
+    if (t.dev == dev && t.base_bits == bits && t.D == D) hit = &t;
+  if (hit && hit->rows >= rows_needed) {
+    *out = hit->ptr;
+    return RA_OK;
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone)
+    return RA_OK;
+  long long n = 4096;
+  while (n < rows_needed) n <<= 1;
+  n = std::min<long long>(n, static_cast<long long>(kTabCacheMaxBytes / row_bytes));
+  float2* ptr = nullptr;
+  if (cudaMalloc(&ptr, static_cast<size_t>(n) * row_bytes) != cudaSuccess) {
+    cudaGetLastError();  // out of memory here is not an error of the call: build per call
+    return RA_OK;
+  }
+  ra::rope_table_kernel<<<grid_for(n * (D / 2), 256, ds->num_sms), 256, 0, s>>>(ptr, 0,
+                                                                                static_cast<int>(n),
+                                                                                D, base);
+  // every stream may read the table once this returns
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) {
+    cudaFree(ptr);
+    return cuda_fail(e, "RoPE table set-up");
+  }
+  if (hit) {
+    g_tabs_retired.push_back(hit->ptr);
+    hit->ptr = ptr;
+    hit->rows = n;
+  } else {
+    g_tabs.push_back(RopeTable{dev, bits, D, n, ptr});
+  }
+  *out = ptr;
+  return RA_OK;
+}
+
 }  // namespace
 
 
@@ -282,16 +351,27 @@ struct PrefillArgs {
 // One launch of the persistent attention kernel: one CTA per SM (fewer when there are fewer
 // work units), each walking its units (query tile, batch, KV group, query-head pair) of the
 // longest-first order in snake order.
+// The launch carries a programmatic dependency on the stream's previous kernel (the key
+// rotation): the kernel's set-up overlaps that kernel's tail and waits on the device before
+// reading anything. Profiled launches go without it, so that the events bracket the kernel.
 ra_status launch_attn(const ra::FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                       const CUtensorMap& tv, int D, int num_sms, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(std::min<long long>(p.n_units, num_sms)));
   const int pi = prof_start(0, s);
-  if (D == 64)
-    ra::attn_fwd_sm100_kernel<64><<<grid, ra::kFwdThreads, ra::FwdCfg<64>::SMEM, s>>>(tq, tk, tv, p);
-  else
-    ra::attn_fwd_sm100_kernel<128><<<grid, ra::kFwdThreads, ra::FwdCfg<128>::SMEM, s>>>(tq, tk, tv, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(ra::kFwdThreads);
+  cfg.dynamicSmemBytes = D == 64 ? ra::FwdCfg<64>::SMEM : ra::FwdCfg<128>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pi < 0 ? 1 : 0;
+  cudaError_t e = D == 64 ? cudaLaunchKernelEx(&cfg, ra::attn_fwd_sm100_kernel<64>, tq, tk, tv, p)
+                          : cudaLaunchKernelEx(&cfg, ra::attn_fwd_sm100_kernel<128>, tq, tk, tv, p);
   prof_stop(0, pi, s);
-  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "attn_fwd launch");
 }
 
@@ -338,22 +418,34 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
   ra_status rs = device_state(&ds);
   if (rs != RA_OK) return rs;
 
-  // workspace: rotated keys (plain prefill only), then the (cos, sin) table for positions
-  // pos_offset + tab_lo .. pos_offset + Sk - 1 (covers every query and new key position)
+  // the (cos, sin) table for positions pos_offset + tab_lo .. pos_offset + Sk - 1 (covers
+  // every query and new key position): from the table cache when the positions allow
   const int tab_lo = std::min(0, Sk - Sq);
   const int tab_len = Sk - tab_lo;
+  const long long tab_pos0 = static_cast<long long>(a.pos_offset) + tab_lo;
+  const float2* tab_cached = nullptr;
+  if (tab_pos0 >= 0) {
+    rs = cached_table(ds, a.rope_base, D, tab_pos0 + tab_len, s, &tab_cached);
+    if (rs != RA_OK) return rs;
+  }
+  // workspace: rotated keys (plain prefill only), then the table when it is not cached
   const size_t krot_bytes = cached ? 0 : (kbytes + 255) & ~static_cast<size_t>(255);
-  const size_t tab_bytes = static_cast<size_t>(tab_len) * (D / 2) * sizeof(float2);
+  const size_t tab_bytes =
+      tab_cached ? 0 : static_cast<size_t>(tab_len) * (D / 2) * sizeof(float2);
   void* ws = nullptr;
-  cudaError_t e = cudaMallocFromPoolAsync(&ws, krot_bytes + tab_bytes, ds->pool, s);
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, std::max<size_t>(krot_bytes + tab_bytes, 256),
+                                          ds->pool, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(workspace)");
   void* k_rot = ws;
-  float2* tab = reinterpret_cast<float2*>(static_cast<char*>(ws) + krot_bytes);
+  const float2* tab = tab_cached ? tab_cached + tab_pos0 * (D / 2)
+                                 : reinterpret_cast<float2*>(static_cast<char*>(ws) + krot_bytes);
 
-  // angles -> (cos, sin) table; then K -> K' once (into the cache, with V, when cached)
-  ra::rope_table_kernel<<<grid_for(static_cast<long long>(tab_len) * (D / 2), 256, ds->num_sms),
-                          256, 0, s>>>(tab, static_cast<long long>(a.pos_offset) + tab_lo, tab_len,
-                                       D, a.rope_base);
+  // angles -> (cos, sin) table (when not cached); then K -> K' once (into the cache, with V,
+  // when cached)
+  if (!tab_cached)
+    ra::rope_table_kernel<<<grid_for(static_cast<long long>(tab_len) * (D / 2), 256,
+                                     ds->num_sms), 256, 0, s>>>(
+        const_cast<float2*>(tab), tab_pos0, tab_len, D, a.rope_base);
   const long long krows = static_cast<long long>(B) * Hkv * Sk;
   if (cached)
     ra::cache_write_kernel<<<grid_for(krows * (D / 8), 256, ds->num_sms), 256, 0, s>>>(
@@ -391,6 +483,7 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.window = a.window;
     p.q_tab_off = (Sk - Sq) - tab_lo;
     p.q_split = Sq;
+    p.q_tab_off2 = p.q_tab_off;
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
     p.rope_base = a.rope_base;
     p.o_acc = nullptr;
@@ -479,20 +572,28 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   DeviceState* ds = nullptr;
   ra_status rs = device_state(&ds);
   if (rs != RA_OK) return rs;
-  // workspace: the (cos, sin) table of the query rows' positions, one table row per query
-  // row (the keys arrive rotated)
-  const size_t tab_bytes = static_cast<size_t>(Sq) * (D / 2) * sizeof(float2);
+  // the (cos, sin) table of the query rows' positions (the keys arrive rotated): the cached
+  // table of absolute positions, else one built here with one row per query row
+  const int n0 = two_seg ? a.q_split : Sq;
+  const long long rows_needed =
+      std::max<long long>(static_cast<long long>(a.q_pos0) + n0,
+                          two_seg ? static_cast<long long>(a.q_pos1) + (Sq - n0) : 0);
+  const float2* tab_cached = nullptr;
+  rs = cached_table(ds, a.rope_base, D, rows_needed, s, &tab_cached);
+  if (rs != RA_OK) return rs;
+  const size_t tab_bytes = tab_cached ? 256 : static_cast<size_t>(Sq) * (D / 2) * sizeof(float2);
   void* ws = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(&ws, tab_bytes, ds->pool, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(workspace)");
   float2* tab = static_cast<float2*>(ws);
-  const int n0 = two_seg ? a.q_split : Sq;
-  ra::rope_table_kernel<<<grid_for(static_cast<long long>(n0) * (D / 2), 256, ds->num_sms), 256,
-                          0, s>>>(tab, a.q_pos0, n0, D, a.rope_base);
-  if (two_seg)
-    ra::rope_table_kernel<<<grid_for(static_cast<long long>(Sq - n0) * (D / 2), 256,
-                                     ds->num_sms), 256, 0, s>>>(
-        tab + static_cast<size_t>(n0) * (D / 2), a.q_pos1, Sq - n0, D, a.rope_base);
+  if (!tab_cached) {
+    ra::rope_table_kernel<<<grid_for(static_cast<long long>(n0) * (D / 2), 256, ds->num_sms),
+                            256, 0, s>>>(tab, a.q_pos0, n0, D, a.rope_base);
+    if (two_seg)
+      ra::rope_table_kernel<<<grid_for(static_cast<long long>(Sq - n0) * (D / 2), 256,
+                                       ds->num_sms), 256, 0, s>>>(
+          tab + static_cast<size_t>(n0) * (D / 2), a.q_pos1, Sq - n0, D, a.rope_base);
+  }
   CUtensorMap tq, tk, tv;
   rs = make_map(&tq, a.q, D, Sq, bhq, 128, q_rows);
   if (rs == RA_OK) rs = make_map(&tk, a.k_rot, D, Sk, bhk, 128, kv_rows);
@@ -500,7 +601,7 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   if (rs == RA_OK) {
     ra::FwdParams p;
     p.out = static_cast<__nv_bfloat16*>(a.out);
-    p.tab = tab;
+    p.tab = tab_cached ? tab_cached : tab;
     p.status = ds->status;
     p.wait_limit = g_wait_limit.load();
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Sk = Sk;
@@ -512,8 +613,10 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
     p.causal = a.causal ? 1 : 0;
     p.off = a.q_pos0 - a.k_pos0;  // query row i at q_pos0 + i, key j at k_pos0 + j
     p.window = 0;
-    p.q_tab_off = 0;
-    p.q_split = n0;  // table row n0 starts the second segment's positions (Sq: none)
+    // query row i sits at q_pos0 + i, or at q_pos1 + (i - n0) in the second segment
+    p.q_tab_off = tab_cached ? a.q_pos0 : 0;
+    p.q_split = n0;
+    p.q_tab_off2 = tab_cached ? a.q_pos1 - n0 : 0;
     p.scale_log2 = kLog2e / std::sqrt(static_cast<float>(D));
     p.rope_base = a.rope_base;
     p.o_acc = a.o_acc;
