@@ -38,7 +38,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from synthetic import DECODE, LLAMA, LONG, make_inputs  # noqa: E402
+from synthetic import DECODE, LLAMA, LONG, Workload, make_inputs  # noqa: E402
 
 PREFILL_W, DECODE_W = LLAMA, DECODE
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -582,6 +582,19 @@ def next_rows_leg(ra, world, rank, dev, peaks):
         f"{P.name} B{P.B} Hq{P.Hq} Hkv{P.Hkv} S{P.Sq} D{P.D} causal into a {P.Sk + 512}-row cache",
         ms, P.flops(), world, "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s")
     del q, k, v, out, kc, vc
+    # other head groupings at the Llama shape: an odd group size (G = 3, whose units pair
+    # two consecutive query tiles of one head) and multi-query attention (8 query heads on
+    # one key/value head)
+    for key, (Bg, Hqg, Hkvg) in (("gqa_group3_prefill", (4, 24, 8)),
+                                 ("mqa_group8_prefill", (4, 8, 1))):
+        Wg = Workload(f"{P.name} G{Hqg // Hkvg}", Bg, Hqg, Hkvg, P.Sq, P.Sk, P.D, P.rope_base)
+        q, k, v = (t.to(dev) for t in make_inputs(Wg, rank_seed(rank, 3)))
+        out = torch.empty_like(q)
+        ms = time_calls(lambda: ra.rope_attn_fwd(q, k, v, Wg.rope_base, 0, True, out=out), 20)
+        res[key] = _rate_entry(
+            f"causal prefill B{Bg} Hq{Hqg} Hkv{Hkvg} (G = {Hqg // Hkvg}) S{P.Sq} D{P.D}", ms,
+            Wg.flops(), world, "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s")
+        del q, k, v, out
     # decode step with append at per-sequence positions, contiguous and paged
     Dw = DECODE_W
     q, kc, vc, kn, vn, pos, pos_h, table = decode_step_inputs(Dw, rank, dev)

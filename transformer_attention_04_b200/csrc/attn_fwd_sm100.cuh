@@ -13,9 +13,11 @@
 // "Transformer Architecture: FlashAttention & RoPE" (KWAS Academy, "Line-by-Line
 // Technical Breakdown") describe.
 //
-// Persistent kernel: one CTA per SM walks a list of work units. A unit is up to two 128-row
-// query tiles ("slots") that share every K/V tile: two query heads of the same KV group at
-// the same positions (GQA with an even group size) or, for odd group sizes, a single tile.
+// Persistent kernel: one CTA per SM walks a list of work units. A unit is two 128-row query
+// tiles ("slots") that share every K/V tile: two query heads of the same KV group at the
+// same positions (GQA with an even group size), or, for odd group sizes (MHA included), two
+// consecutive query tiles of one head (the first tile's rows see one more key tile than
+// they may, which the causal mask zeroes).
 // Units are ordered longest causal extent first and dealt to the CTAs in snake order
 // (round k runs forward over the CTAs when k is even, backward when odd), which balances the
 // causal triangle. Warp roles (384 threads):
@@ -56,7 +58,9 @@ struct FwdParams {
   int B, Hq, Hkv, Sq, Sk;
   int G;                // Hq / Hkv
   int n_slots;          // query tiles per unit (1 or 2)
-  int ppg;              // units per (batch, KV group, query tile) = G / n_slots
+  int pair_q;           // 1: the slots are two consecutive query tiles of one head (odd G);
+                        // 0: the same query tile of two heads of the KV group (even G)
+  int ppg;              // units per (batch, KV group, query-tile group)
   int n_qtiles;         // ceil(Sq / 128)
   int n_units;          // n_qtiles * B * Hkv * ppg
   int causal;
@@ -108,26 +112,32 @@ struct FwdCfg {
   static_assert(SMEM <= 232448, "shared memory per block");
 };
 
-// One work unit: which query tile(s), heads and KV tiles.
+// One work unit: which query tile(s), heads and KV tiles. Slot s holds query rows
+// q0 + dq(s) .. + 127 of head h0 + dh(s).
 struct Unit {
   int b, h0, kv_bh, q0, j_lo, n_it;
 };
+__device__ __forceinline__ int slot_dq(const FwdParams& p, int s) { return p.pair_q ? 128 * s : 0; }
+__device__ __forceinline__ int slot_dh(const FwdParams& p, int s) { return p.pair_q ? 0 : s; }
 
-// Unit u of the longest-first order: rank t of the query tiles (causal: tile n_qtiles-1-t),
-// then batch, KV group and head pair.
+// Unit u of the longest-first order: rank t of the query-tile groups (one tile, or two
+// consecutive tiles with pair_q; causal: the last group first), then batch, KV group and
+// head (pair).
 __device__ __forceinline__ Unit unit_at(const FwdParams& p, int u) {
   Unit w;
   const int per_tile = p.B * p.Hkv * p.ppg;
   const int t_rank = u / per_tile;
   const int rem = u - t_rank * per_tile;
-  const int qt = p.causal ? (p.n_qtiles - 1 - t_rank) : t_rank;
+  const int n_groups = p.pair_q ? (p.n_qtiles + 1) / 2 : p.n_qtiles;
+  const int qg = p.causal ? (n_groups - 1 - t_rank) : t_rank;
   w.b = rem / (p.Hkv * p.ppg);
   const int g = (rem / p.ppg) % p.Hkv;
-  w.h0 = g * p.G + (rem % p.ppg) * p.n_slots;
+  w.h0 = g * p.G + (rem % p.ppg) * (p.pair_q ? 1 : p.n_slots);
   w.kv_bh = w.b * p.Hkv + g;
-  w.q0 = qt * 128;
+  w.q0 = qg * 128 * (p.pair_q ? 2 : 1);
+  const int q_last = w.q0 + slot_dq(p, p.n_slots - 1) + 127;  // the unit's last query row
   int n_kv = (p.Sk + 127) / 128;
-  if (p.causal) n_kv = min(n_kv, (min(p.Sq - 1, w.q0 + 127) + p.off) / 128 + 1);
+  if (p.causal) n_kv = min(n_kv, (min(p.Sq - 1, q_last) + p.off) / 128 + 1);
   // with a sliding window, tiles wholly below the first row's window are skipped too
   w.j_lo = (p.window > 0) ? max(0, w.q0 + p.off - p.window + 1) / 128 : 0;
   w.n_it = n_kv - w.j_lo;  // KV tiles visited: j_lo .. n_kv - 1
@@ -254,8 +264,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_expect_tx(bar(C::B_QFULL + qb), ns * C::TILE);
         for (int s = 0; s < ns; ++s)
           for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_3d_hint(sQ + (qb * 2 + s) * C::TILE + kb * C::BLK, &tm_q, kb * 64, w.q0,
-                             w.b * p.Hq + w.h0 + s, bar(C::B_QFULL + qb), pol_once);
+            tma_load_3d_hint(sQ + (qb * 2 + s) * C::TILE + kb * C::BLK, &tm_q, kb * 64,
+                             w.q0 + slot_dq(p, s), w.b * p.Hq + w.h0 + slot_dh(p, s),
+                             bar(C::B_QFULL + qb), pol_once);
         if (qb) ++q_issued1; else ++q_issued0;
         return true;
       };
@@ -435,10 +446,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         return false;
       const Unit w = unit_at(p, u);
       const int kb = ck >> 3, c = ck & 7;
+      // slots at the same positions (two heads) share one pass; paired query tiles take one
+      // pass each
+      const int per_pass = p.pair_q ? 1 : ns;
+      for (int s0 = 0; s0 < ns; s0 += per_pass) {
       float2 cs[4];
 #pragma unroll 1
       for (int rr = 0; rr < RB; ++rr) {
-        const int row = rb0 + rr, qr = w.q0 + row;
+        const int row = rb0 + rr, qr = w.q0 + slot_dq(p, s0) + row;
         if (qr >= p.Sq) break;
         if (rr == 0 || qr == p.q_split) {
           const int trow = (qr < p.q_split ? p.q_tab_off : p.q_tab_off2) + qr;
@@ -456,10 +471,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 cs[e].y * step[e].x + cs[e].x * step[e].y);
         }
         const uint32_t off = kb * C::BLK + row * 128 + ((c ^ (row & 7)) << 4);
-        for (int s = 0; s < ns; ++s) {
+        for (int s = s0; s < s0 + per_pass; ++s) {
           uint4* ptr = reinterpret_cast<uint4*>(smem + C::OFF_Q + (qb * 2 + s) * C::TILE + off);
           *ptr = rotate8(*ptr, cs);
         }
+      }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -484,7 +500,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     int t = 0;  // global tile counter
     for (int k = 0; ok && unit_of(p, k) >= 0; ++k) {
       const Unit w = unit_at(p, unit_of(p, k));
-      const int qrow = w.q0 + r;
+      const int q0s = w.q0 + slot_dq(p, s);  // this slot's first query row
+      const int qrow = q0s + r;
+      const int head = w.h0 + slot_dh(p, s);
       float m = -INFINITY;  // running row max, in log2 units of the scaled score
       float l = 0.f;        // running row sum of 2^(x - m)
       const int lim_causal = min(p.Sk - 1, qrow + p.off);
@@ -504,8 +522,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         // causal / window / sequence-end mask, only on tiles that reach past some row's limit
         const int kbase = (w.j_lo + jj) * 128;
         const bool need_mask = (kbase + 128 > p.Sk) ||
-                               (p.causal && kbase + 127 > w.q0 + p.off) ||
-                               (p.window > 0 && kbase + p.window < w.q0 + 128 + p.off);
+                               (p.causal && kbase + 127 > q0s + p.off) ||
+                               (p.window > 0 && kbase + p.window < q0s + 128 + p.off);
         if (need_mask) {
           const int lim_k = (p.causal ? lim_causal : p.Sk - 1) - kbase;
           const int lo_k = (p.window > 0) ? qrow + p.off - p.window + 1 - kbase : 0;
@@ -585,7 +603,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (p.o_acc != nullptr) {
         // partial mode: O / l and the LSE in fp32, merged with the running result
         // (weights exp(lse - merged lse) on each side); every row has at least one allowed key
-        const long long row = static_cast<long long>(w.b * p.Hq + w.h0 + s) * p.acc_rows + qrow;
+        const long long row = static_cast<long long>(w.b * p.Hq + head) * p.acc_rows + qrow;
         const float lse_new = (m + log2f(l)) * kLn2;
         float w_old = 0.f, w_new = 1.0f / l, lse_out = lse_new;
         if (p.accumulate && qrow < p.Sq) {
@@ -640,7 +658,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float inv = 1.0f / l;
         const uint64_t pol_out = l2_policy_evict_first();
         __nv_bfloat16* orow =
-            p.out + (static_cast<long long>(w.b * p.Hq + w.h0 + s) * p.Sq + qrow) * D;
+            p.out + (static_cast<long long>(w.b * p.Hq + head) * p.Sq + qrow) * D;
 #pragma unroll
         for (int cb = 0; cb < D; cb += 32) {
           uint32_t o[32];

@@ -408,9 +408,13 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     if (overlap(a.k_cache, cbytes, a.v_cache, cbytes)) return RA_ERR_INVALID_ARG;
   }
   const int G = Hq / Hkv;
-  const int n_slots = (G % 2 == 0) ? 2 : 1;
+  // two slots per unit: two heads of a KV group (even G) or two consecutive query tiles of
+  // one head (odd G)
+  const int pair_q = G % 2;
   const int n_qtiles = (Sq + 127) / 128;
-  const long long n_units = static_cast<long long>(n_qtiles) * B * Hkv * (G / n_slots);
+  const int ppg = pair_q ? G : G / 2;
+  const long long n_units =
+      static_cast<long long>(pair_q ? (n_qtiles + 1) / 2 : n_qtiles) * B * Hkv * ppg;
   if (n_units > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL)
     return RA_ERR_UNSUPPORTED;
 
@@ -474,8 +478,9 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.wait_limit = g_wait_limit.load();
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Sk = static_cast<int>(T);
     p.G = G;
-    p.n_slots = n_slots;
-    p.ppg = G / n_slots;
+    p.n_slots = 2;
+    p.pair_q = pair_q;
+    p.ppg = ppg;
     p.n_qtiles = n_qtiles;
     p.n_units = static_cast<int>(n_units);
     p.causal = a.causal ? 1 : 0;
@@ -563,9 +568,13 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
                  overlap(a.out, outbytes, a.lse_acc, lbytes))))
     return RA_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
-  const int n_slots = (G % 2 == 0) ? 2 : 1;
+  // two slots per unit: two heads of a KV group (even G) or two consecutive query tiles of
+  // one head (odd G)
+  const int pair_q = G % 2;
   const int n_qtiles = (Sq + 127) / 128;
-  const long long n_units = static_cast<long long>(n_qtiles) * B * Hkv * (G / n_slots);
+  const int ppg = pair_q ? G : G / 2;
+  const long long n_units =
+      static_cast<long long>(pair_q ? (n_qtiles + 1) / 2 : n_qtiles) * B * Hkv * ppg;
   if (n_units > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL)
     return RA_ERR_UNSUPPORTED;
 
@@ -606,8 +615,9 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
     p.wait_limit = g_wait_limit.load();
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Sk = Sk;
     p.G = G;
-    p.n_slots = n_slots;
-    p.ppg = G / n_slots;
+    p.n_slots = 2;
+    p.pair_q = pair_q;
+    p.ppg = ppg;
     p.n_qtiles = n_qtiles;
     p.n_units = static_cast<int>(n_units);
     p.causal = a.causal ? 1 : 0;
