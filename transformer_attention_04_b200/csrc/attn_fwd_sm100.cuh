@@ -538,10 +538,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         // P with the new reference). Either way every row ends with the same values as the
         // plain max-first order.
         float rs = 0.f;
-        bool done = false;
+        bool done = false, spec = false;
         float mt = -INFINITY;
         if (!__any_sync(0xffffffffu, m == -INFINITY)) {
           rs = softmax_p_store(sr, sl2, m, tS);
+          spec = true;
           // every p <= 2^8 unless the tile's row sum exceeds 2^8 (or is inf / NaN)
           done = !__any_sync(0xffffffffu, !(rs <= 256.0f));
         }
@@ -582,9 +583,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
           }
           // p = 2^(s * log2(e)/sqrt(D) - m) -> bf16 P over the S columns; a row that has seen
-          // no allowed key yet (only under a window) keeps m = -inf and gets P = 0
-          const float m_use = (m == -INFINITY) ? 0.f : m;
-          rs = softmax_p_store(sr, sl2, m_use, tS);
+          // no allowed key yet (only under a window) keeps m = -inf and gets P = 0. A
+          // speculative P whose reference no row of the warp moved is already that P: a row
+          // whose reference came from a few keys (a window's first tile) often sums past 2^8
+          // without its max growing by 8.
+          if (!spec || __any_sync(0xffffffffu, upd)) {
+            const float m_use = (m == -INFINITY) ? 0.f : m;
+            rs = softmax_p_store(sr, sl2, m_use, tS);
+          }
         }
         l += rs;
         tmem_wait_st();
