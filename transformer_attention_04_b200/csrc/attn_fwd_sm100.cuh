@@ -395,12 +395,13 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             tc_fence_after();
             issue_pv(1, slot(2 * t + 1), jj > 0);
             if (last) umma_commit(bar(C::B_OFULL + 1));
+            umma_commit(bar(C::B_EMPTY + slot(2 * t + 1)));
             if (has_next) {
               issue_s(qbn * 2 + 1, 1, slot(2 * t + 2));
               umma_commit(bar(C::B_SFULL + 1));
             }
           }
-          umma_commit(bar(C::B_EMPTY + slot(2 * t + 1)));
+          if (ns == 1) umma_commit(bar(C::B_EMPTY + slot(2 * t + 1)));
           if (has_next) {
             if (next_last) umma_commit(bar(C::B_QEMPTY + qbn));  // that unit's last S
             umma_commit(bar(C::B_EMPTY + slot(2 * t + 2)));
