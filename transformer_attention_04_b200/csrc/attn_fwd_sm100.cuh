@@ -528,9 +528,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (need_mask) {
           const int lim_k = (p.causal ? lim_causal : p.Sk - 1) - kbase;
           const int lo_k = (p.window > 0) ? qrow + p.off - p.window + 1 - kbase : 0;
+          // the sign of (lim_k - c) | (c - lo_k) masks the element: integer ops, no branch or
+          // predicate (the limits differ from lane to lane)
+          if (p.window > 0) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > lim_k || c < lo_k) sr[c] = 0xff800000u;  // -inf
+            for (int c = 0; c < 128; ++c) {
+              const uint32_t mk = static_cast<uint32_t>(((lim_k - c) | (c - lo_k)) >> 31);
+              sr[c] = (sr[c] & ~mk) | (0xff800000u & mk);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+              const uint32_t mk = static_cast<uint32_t>((lim_k - c) >> 31);
+              sr[c] = (sr[c] & ~mk) | (0xff800000u & mk);
+            }
+          }
         }
         // online softmax with a lazily updated reference max m. Once a row has a
         // reference, P is computed speculatively with it; every p is then at most 2^8 unless
