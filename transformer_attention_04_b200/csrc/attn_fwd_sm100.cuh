@@ -27,7 +27,9 @@
 //   warps 2-3     RoPE rotation of each unit's Q tiles in shared memory, done while the
 //                 previous unit runs.
 //   warps 4-7     softmax warpgroup of slot 0 (thread = query row = TMEM lane); after a
-//                 unit's last tile it writes the unit's output from TMEM.
+//                 unit's last tile it writes the unit's output from TMEM into the slot's
+//                 finished Q tile in shared memory, and one of its threads stores the tile
+//                 with TMA (an fp32 merge into the running result in partial mode).
 //   warps 8-11    softmax warpgroup of slot 1.
 // Per KV tile j the issuer runs S_s = Q_s K_j^T (SS MMA, fp32 in TMEM), the softmax group
 // turns S_s into bf16 P_s written over the same TMEM columns, and the issuer runs
@@ -105,7 +107,10 @@ struct FwdCfg {
       B_SFULL = 6,                     // [s]: S_s in TMEM
       B_PFULL = 8,                     // [s]: P_s in TMEM (4 softmax warps)
       B_OFULL = 10,                    // [s]: the unit's last PV_s done
-      B_DRAIN = 12, B_FULL = 13, B_EMPTY = 13 + NSLOT, N_BAR = 13 + 2 * NSLOT;
+      B_DRAIN = 12,
+      B_QSTAGED = 13,                  // [b]: the unit's outputs, staged in its Q tiles, stored
+      B_EPI = 15,                      // [s]: slot s's rows staged (4 softmax warps)
+      B_FULL = 17, B_EMPTY = 17 + NSLOT, N_BAR = 17 + 2 * NSLOT;
   static constexpr int OFF_TMEM_SLOT = 8 * N_BAR;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
   static_assert(OFF_ABORT + 4 <= 512, "barrier area");
@@ -185,7 +190,8 @@ template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
@@ -211,6 +217,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(C::B_SFULL + i), 1);
       mbar_init(bar(C::B_PFULL + i), 4);   // one arrival per softmax warp
       mbar_init(bar(C::B_OFULL + i), 1);
+      mbar_init(bar(C::B_QSTAGED + i), ns);  // one TMA store per slot
+      mbar_init(bar(C::B_EPI + i), 4);
     }
     mbar_init(bar(C::B_DRAIN), 1);
     for (int i = 0; i < C::NSLOT; ++i) {
@@ -259,6 +267,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         // the buffer's previous unit (k - 2) must have issued its last S
         if (k >= 2 && !mbar_wait(bar(C::B_QEMPTY + qb), ((k - 2) >> 1) & 1, lim, abort_flag,
                                  p.status))
+          return false;
+        // (plain mode) unit k - 2's outputs were staged in this buffer: their store has read it
+        if (k >= 2 && p.o_acc == nullptr &&
+            !mbar_wait(bar(C::B_QSTAGED + qb), ((k - 2) >> 1) & 1, lim, abort_flag, p.status))
           return false;
         const Unit w = unit_at(p, u);
         mbar_expect_tx(bar(C::B_QFULL + qb), ns * C::TILE);
@@ -673,35 +685,55 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (qrow < p.Sq) p.lse_acc[row] = lse_out;
       } else {
-        // O / l -> bf16
+        // O / l -> bf16, written row by row into this slot's Q tile of the unit (no MMA reads
+        // it any more: OFULL follows the unit's last S_s) in the 128-byte swizzled layout of
+        // the output's tensor map; then one thread stores the tile with TMA (rows past Sq are
+        // clipped by the map) and releases the buffer to the producer.
         const float inv = 1.0f / l;
-        const uint64_t pol_out = l2_policy_evict_first();
-        __nv_bfloat16* orow =
-            p.out + (static_cast<long long>(w.b * p.Hq + head) * p.Sq + qrow) * D;
+        const int qb = k & 1;
+        uint8_t* stage = smem + C::OFF_Q + (qb * 2 + s) * C::TILE;
 #pragma unroll
         for (int cb = 0; cb < D; cb += 32) {
           uint32_t o[32];
           tmem_ld32(tO + cb, o);
           tmem_wait_ld();
-          if (qrow < p.Sq) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + cb);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
-              v.y = pack_bf16(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
-              v.z = pack_bf16(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
-              v.w = pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
-              st_global_v4_hint(dst + e, v, pol_out);
-            }
+          for (int e = 0; e < 4; ++e) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+            const int ch = (cb & 63) / 8 + e;  // 16-byte chunk within the 64-column block
+            *reinterpret_cast<uint4*>(stage + (cb >> 6) * C::BLK + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_EPI + s));
+        if (qd == 0 && lane == 0) {
+          if (!mbar_wait(bar(C::B_EPI + s), k & 1, lim, abort_flag, p.status)) {
+            ok = false;
+          } else {
+            if (w.q0 + slot_dq(p, s) < p.Sq)  // (the second tile of an odd count has no rows)
+              for (int kb = 0; kb < C::KB; ++kb)
+                tma_store_3d(&tm_o, smem_u32(stage + kb * C::BLK), kb * 64, w.q0 + slot_dq(p, s),
+                             w.b * p.Hq + head);
+            bulk_commit_group();
+            bulk_wait_read_all();
+            mbar_arrive(bar(C::B_QSTAGED + qb));
+          }
+        }
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, ok)) break;
       }
       // the next PFULL arrival (after tc_fence_before) orders these TMEM reads before the
       // next unit's first PV_s
     }
   }
   }
+  // the output tiles stored with TMA have been written before the CTA exits
+  if (warp >= 4 && (warp & 3) == 0 && lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

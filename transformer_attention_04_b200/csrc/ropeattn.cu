@@ -355,7 +355,8 @@ struct PrefillArgs {
 // rotation): the kernel's set-up overlaps that kernel's tail and waits on the device before
 // reading anything. Profiled launches go without it, so that the events bracket the kernel.
 ra_status launch_attn(const ra::FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                      const CUtensorMap& tv, int D, int num_sms, cudaStream_t s) {
+                      const CUtensorMap& tv, const CUtensorMap& to, int D, int num_sms,
+                      cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(std::min<long long>(p.n_units, num_sms)));
   const int pi = prof_start(0, s);
   cudaLaunchConfig_t cfg = {};
@@ -368,8 +369,9 @@ ra_status launch_attn(const ra::FwdParams& p, const CUtensorMap& tq, const CUten
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pi < 0 ? 1 : 0;
-  cudaError_t e = D == 64 ? cudaLaunchKernelEx(&cfg, ra::attn_fwd_sm100_kernel<64>, tq, tk, tv, p)
-                          : cudaLaunchKernelEx(&cfg, ra::attn_fwd_sm100_kernel<128>, tq, tk, tv, p);
+  cudaError_t e =
+      D == 64 ? cudaLaunchKernelEx(&cfg, ra::attn_fwd_sm100_kernel<64>, tq, tk, tv, to, p)
+              : cudaLaunchKernelEx(&cfg, ra::attn_fwd_sm100_kernel<128>, tq, tk, tv, to, p);
   prof_stop(0, pi, s);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "attn_fwd launch");
@@ -461,9 +463,11 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
         static_cast<const uint4*>(a.k), static_cast<uint4*>(k_rot), tab, krows, Sk, D, 0, -tab_lo,
         a.rope_base, Sk, Sk);
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const long long bkv = static_cast<long long>(B) * Hkv;
   rs = make_map(&tq, a.q, D, Sq, static_cast<long long>(B) * Hq, 128);
+  // the output tiles leave through shared memory with TMA, in Q's geometry
+  if (rs == RA_OK) rs = make_map(&to, a.out, D, Sq, static_cast<long long>(B) * Hq, 128);
   if (rs == RA_OK)
     rs = cached ? make_map(&tk, a.k_cache, D, static_cast<int>(T), bkv, 128, a.S_cache)
                 : make_map(&tk, k_rot, D, Sk, bkv, 128);
@@ -495,7 +499,7 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.lse_acc = nullptr;
     p.accumulate = 0;
     p.acc_rows = Sq;
-    rs = launch_attn(p, tq, tk, tv, D, ds->num_sms, s);
+    rs = launch_attn(p, tq, tk, tv, to, D, ds->num_sms, s);
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
   if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
@@ -633,7 +637,7 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
     p.lse_acc = a.lse_acc;
     p.accumulate = a.accumulate ? 1 : 0;
     p.acc_rows = acc_rows;
-    rs = launch_attn(p, tq, tk, tv, D, ds->num_sms, s);
+    rs = launch_attn(p, tq, tk, tv, tq, D, ds->num_sms, s);  // partial mode: no output map
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
   if (rs == RA_OK && ef != cudaSuccess) rs = cuda_fail(ef, "cudaFreeAsync(workspace)");
