@@ -87,9 +87,16 @@ RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void
  *   k_rot  [B, Hkv, Sk, D] bf16 (read), keys already rotated to k_pos0 + j (for example by
  *          rope_attn_rotate with pos_offset = k_pos0).   v [B, Hkv, Sk, D] bf16 (read).
  *   o_acc  [B, Hq, Sq, D] fp32 and lse_acc [B, Hq, Sq] fp32 (natural log): the running
- *          result, normalised (O, not O times the sum). accumulate == 0: overwritten with
- *          this block's result. accumulate != 0: merged with their contents; an lse_acc
- *          entry of -inf marks an empty accumulator row.
+ *          result, normalised (O, not O times the sum).
+ *   accumulate: bit RA_PARTIAL_ACCUMULATE clear: o_acc / lse_acc are overwritten with this
+ *          block's result; set: merged with their contents (an lse_acc entry of -inf marks an
+ *          empty accumulator row). Bit RA_PARTIAL_CHAINED: the caller guarantees that q,
+ *          k_rot and v were complete before the previous kernel on the stream started (for
+ *          example consecutive blocks of a ring whose keys were rotated before the first
+ *          block). The launch then runs alongside that kernel's last wave and waits for it
+ *          only before merging into o_acc / lse_acc / out. Without the guarantee the bit
+ *          gives wrong results; leave it clear on a block that follows the kernel which
+ *          produced its inputs.
  *   out    [B, Hq, Sq, D] bf16 or NULL: when given, also receives the merged result
  *          (pass it on the last block).
  *   causal: key j is allowed to query row i iff k_pos0 + j <= q_pos0 + i; requires
@@ -110,6 +117,8 @@ RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void
  * the Sq query positions). Returns RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED or
  * RA_ERR_CUDA.
  */
+#define RA_PARTIAL_ACCUMULATE 1
+#define RA_PARTIAL_CHAINED 2
 RA_API ra_status rope_attn_fwd_partial(const void* q, const void* k_rot, const void* v,
                                        float* o_acc, float* lse_acc, void* out, int B, int Hq,
                                        int Hkv, int Sq, int Sk, int D, float rope_base,

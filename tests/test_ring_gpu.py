@@ -115,6 +115,34 @@ def test_partial_merge_of_key_ranges(D, split):
         _check_lse(lse, want_l, "merged lse")
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_partial_chained_blocks(D):
+    # consecutive blocks whose keys were all rotated before the first call, launched with the
+    # chained flag: each may run alongside its predecessor and waits for it only before its
+    # merge. The merged result must equal the block over all keys.
+    B, Hq, Hkv, Sq, Sk, qp, nb = 2, 16, 4, 1024, 2048, 4096, 4
+    base = 500000.0
+    q, k, v = _bf16((B, Hq, Sq, D), 31), _bf16((B, Hkv, Sk, D), 32), _bf16((B, Hkv, Sk, D), 33)
+    kr = _rotated_keys(k, 0, base)
+    want_o, want_l = oracle.rope_attn_fwd_partial(to_f64(q), to_f64(kr), to_f64(v), base, qp, 0,
+                                                  True)
+    qg, krg, vg = q.cuda(), kr.cuda(), v.cuda()
+    L = Sk // nb
+    blocks = [(krg[:, :, i * L:(i + 1) * L].contiguous(), vg[:, :, i * L:(i + 1) * L].contiguous())
+              for i in range(nb)]
+    o_acc = torch.full((B, Hq, Sq, D), float("nan"), device="cuda")
+    lse = torch.full((B, Hq, Sq), float("nan"), device="cuda")
+    out = torch.empty((B, Hq, Sq, D), device="cuda", dtype=torch.bfloat16)
+    for i, (kk, vv) in enumerate(blocks):
+        ra.rope_attn_fwd_partial(qg, kk, vv, o_acc, lse, base, qp, i * L, True,
+                                 accumulate=i > 0, out=out if i == nb - 1 else None,
+                                 chained=i > 0)
+    _ok()
+    assert_parity(o_acc, want_o, f"chained o_acc D{D}")
+    assert_parity(out, want_o, f"chained out D{D}")
+    _check_lse(lse, want_l, f"chained lse D{D}")
+
+
 def test_partial_merge_into_empty_accumulator_rows():
     # an lse_acc of -inf marks an empty row: merging into it takes the block as it is
     B, Hq, Hkv, S, D = 1, 4, 2, 160, 128

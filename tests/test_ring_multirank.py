@@ -51,7 +51,7 @@ def _worker(rank, world, port, causal, q_out, layout="contiguous"):
         return out
 
     def cpu_partial(q, k_rot, v, o_acc, lse_acc, rope_base, q_pos0, k_pos0, causal=True,
-                    accumulate=False, out=None, q_split=0, q_pos1=0):
+                    accumulate=False, out=None, q_split=0, q_pos1=0, chained=False):
         calls.append((q_pos0, k_pos0, bool(accumulate), out is not None))
         if 0 < q_split < q.shape[2]:
             # two query segments (unmasked): each row's result depends only on its position

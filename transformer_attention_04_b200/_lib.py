@@ -179,13 +179,16 @@ def _head_rows(t, name, dtype, shape):
 
 def rope_attn_fwd_partial(q, k_rot, v, o_acc, lse_acc, rope_base: float, q_pos0: int,
                           k_pos0: int, causal: bool = True, accumulate: bool = False, out=None,
-                          q_split: int = 0, q_pos1: int = 0, stream=None):
+                          q_split: int = 0, q_pos1: int = 0, stream=None, chained: bool = False):
     """One ring-attention block: q [B,Hq,Sq,D] (rotated here to q_pos0+i; rows >= q_split at
     q_pos1 + (i - q_split) when 0 < q_split < Sq, unmasked calls only) against keys k_rot
     [B,Hkv,Sk,D] already rotated to k_pos0+j, and v. The block's normalised output and
     natural-log LSE go to o_acc [B,Hq,Sq,D] / lse_acc [B,Hq,Sq] (fp32), merged with their
     contents when ``accumulate``; ``out`` (bf16), if given, also receives the merged result.
-    Every tensor may be a slice along the sequence axis of a longer one (q[:, :, a:b])."""
+    Every tensor may be a slice along the sequence axis of a longer one (q[:, :, a:b]).
+    ``chained``: q, k_rot and v were complete before the previous kernel on the stream
+    started (consecutive ring blocks whose keys were rotated up front); the block then runs
+    alongside that kernel and waits for it only before its merge."""
     if q.dim() != 4 or k_rot.dim() != 4:
         raise ValueError("q, k_rot, v must be 4-D [B, H, S, D]")
     B, Hq, Sq, D = q.shape
@@ -205,7 +208,8 @@ def rope_attn_fwd_partial(q, k_rot, v, o_acc, lse_acc, rope_base: float, q_pos0:
     st = lib().rope_attn_fwd_partial(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(),
                                      o_acc.data_ptr(), lse_acc.data_ptr(), o, B, Hq, Hkv, Sq, Sk,
                                      D, float(rope_base), int(q_pos0), int(k_pos0),
-                                     int(bool(causal)), int(bool(accumulate)), q_rows, kv_rows,
+                                     int(bool(causal)),
+                                     (1 if accumulate else 0) | (2 if chained else 0), q_rows, kv_rows,
                                      acc_rows, int(q_split), int(q_pos1), _stream(stream))
     _raise(st, "rope_attn_fwd_partial")
     return out

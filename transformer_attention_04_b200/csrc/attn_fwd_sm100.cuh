@@ -80,6 +80,8 @@ struct FwdParams {
   float* lse_acc;
   int accumulate;
   int acc_rows;  // partial mode: rows between heads in o_acc / lse_acc / out (>= Sq)
+  int dep_late;  // partial mode: the inputs were complete before the previous kernel started;
+                 // wait for that kernel only before merging into the running result
 };
 
 template <int D>
@@ -242,8 +244,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // launched behind the key rotation with a programmatic dependency: the set-up above overlaps
-  // its tail, the rotated keys and the table are read only after it has completed
-  grid_dep_wait();
+  // its tail, the rotated keys and the table are read only after it has completed. A chained
+  // ring block (dep_late) reads only inputs that were complete before that kernel started and
+  // waits before its first merge instead. Either way the next launch may start its set-up.
+  if (!p.dep_late) grid_dep_wait();
+  grid_dep_launch();
 
   // Register split: launched at 168 per thread (384 x 168 = 64512); the control
   // warpgroup gives back to 80, the two softmax warpgroups take 208
@@ -632,6 +637,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       tc_fence_after();
       if (p.o_acc != nullptr) {
+        if (p.dep_late) grid_dep_wait();  // the previous kernel's merges are complete
         // partial mode: O / l and the LSE in fp32, merged with the running result
         // (weights exp(lse - merged lse) on each side); every row has at least one allowed key
         const long long row = static_cast<long long>(w.b * p.Hq + head) * p.acc_rows + qrow;

@@ -499,6 +499,7 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.lse_acc = nullptr;
     p.accumulate = 0;
     p.acc_rows = Sq;
+    p.dep_late = 0;
     rs = launch_attn(p, tq, tk, tv, to, D, ds->num_sms, s);
   }
   cudaError_t ef = cudaFreeAsync(ws, s);
@@ -635,7 +636,8 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
     p.rope_base = a.rope_base;
     p.o_acc = a.o_acc;
     p.lse_acc = a.lse_acc;
-    p.accumulate = a.accumulate ? 1 : 0;
+    p.accumulate = (a.accumulate & RA_PARTIAL_ACCUMULATE) ? 1 : 0;
+    p.dep_late = (a.accumulate & RA_PARTIAL_CHAINED) ? 1 : 0;
     p.acc_rows = acc_rows;
     rs = launch_attn(p, tq, tk, tv, tq, D, ds->num_sms, s);  // partial mode: no output map
   }

@@ -69,8 +69,9 @@ def zigzag_calls(rank: int, world: int, causal: bool):
 
 
 def _zigzag_issue(partial_fn, calls, i, rank, world, c, q, k_cur, v_cur, acc_o, acc_l, out,
-                  rope_base):
-    """Launch call i of zigzag_calls on the views it names."""
+                  rope_base, chained=False):
+    """Launch call i of zigzag_calls on the views it names. ``chained``: its inputs were
+    complete before the previous kernel on the stream started (see rope_attn_fwd_partial)."""
     t, src, qh, kh, masked = calls[i]
     sl = {"lo": slice(0, c), "hi": slice(c, 2 * c), "all": slice(0, 2 * c)}
 
@@ -93,7 +94,7 @@ def _zigzag_issue(partial_fn, calls, i, rank, world, c, q, k_cur, v_cur, acc_o, 
     partial_fn(q[:, :, sl[qh]], k_cur[:, :, sl[kh]], v_cur[:, :, sl[kh]], acc_o[:, :, sl[qh]],
                acc_l[:, :, sl[qh]], rope_base, q_pos0, k_pos0, causal=masked,
                accumulate=all(written.values()), out=out[:, :, sl[qh]] if last else None,
-               q_split=split, q_pos1=q_pos1)
+               q_split=split, q_pos1=q_pos1, **({"chained": True} if chained else {}))
 
 
 def ring_attention(q, k, v, rope_base: float, causal: bool = True, group=None, out=None, *,
@@ -201,9 +202,14 @@ def _ring_zigzag(q, k, v, rope_base, causal, group, out, world, rank, partial_fn
                    dist.P2POp(dist.irecv, dst[0], prv, group),
                    dist.P2POp(dist.irecv, dst[1], prv, group)]
             reqs = dist.batch_isend_irecv(ops)
+        first_of_step = True
         while i < len(calls) and calls[i][0] == t:
+            # a later call of the same step follows an attention launch whose inputs (and its
+            # own) were ready before it; the first call of a step follows the key rotation or
+            # the wait for the received block
             _zigzag_issue(partial_fn, calls, i, rank, world, c, q, cur[0], cur[1], acc_o, acc_l,
-                          out, rope_base)
+                          out, rope_base, chained=not first_of_step)
+            first_of_step = False
             i += 1
         for r in reqs:
             r.wait()
@@ -246,10 +252,13 @@ def ring_attention_local(q, k, v, rope_base: float, n_ranks: int, causal: bool =
             on_rank(r, "start")
         used = [(t, src) for t, src, u in ring_steps(r, n_ranks, causal) if u]
         for i, (_, src) in enumerate(used):
+            # every block after the very first follows an attention launch, and all keys were
+            # rotated before the first: it may run alongside its predecessor's last wave
             _lib.rope_attn_fwd_partial(qs[r], blocks[src][0], blocks[src][1], o_acc, lse_acc,
                                        rope_base, r * L, src * L, causal=causal,
                                        accumulate=i > 0,
-                                       out=outs[r] if i == len(used) - 1 else None)
+                                       out=outs[r] if i == len(used) - 1 else None,
+                                       chained=r > 0 or i > 0)
         if on_rank:
             on_rank(r, "end")
     return torch.cat(outs, dim=2, out=out) if out is not None else torch.cat(outs, dim=2)
@@ -284,8 +293,9 @@ def _ring_zigzag_local(q, k, v, rope_base, n, causal, out, on_rank):
             on_rank(r, "start")
         calls = zigzag_calls(r, n, causal)
         for i, (_, src, _, _, _) in enumerate(calls):
+            # all keys were rotated before the first call (see ring_attention_local)
             _zigzag_issue(_lib.rope_attn_fwd_partial, calls, i, r, n, c, qs[r], ks[src], vs[src],
-                          acc_o, acc_l, outs[r], rope_base)
+                          acc_o, acc_l, outs[r], rope_base, chained=r > 0 or i > 0)
         if on_rank:
             on_rank(r, "end")
     if out is None:
