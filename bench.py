@@ -395,7 +395,7 @@ def run_ours(args):
                    "roofline": {"bound": "hbm", "achieved": split_gbs, "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": split_gbs / peaks["hbm_gbs"],
                                 "peak_source": peak_src,
-                                "kernel": "decode_split_kernel<128>",
+                                "kernel": "decode_split_kernel<128, false>",
                                 "traffic": recorded_traffic("decode_split_kernel decode")}},
         "prefill_ms_per_call": pre_ms / K,
         # the host's own cost per step: the median over the first steps, which run before

@@ -89,9 +89,17 @@ struct DecCfg {
   static_assert(OFF_WS_ML + 4 * 8 * 8 <= NST * STAGE, "merge scratch");
 };
 
-// byte offset of (key, d) inside one swizzled 64-key x D tile; d a multiple of 8
-__device__ __forceinline__ uint32_t dec_swz(int key, int d) {
-  return static_cast<uint32_t>((d >> 6) * (64 * 128) + key * 128 +
+// Byte offset of (key, d) inside one swizzled 64-key x D tile; d a multiple of 8. The tile is
+// cut into groups of 2^lp keys (one page of a paged pool, or all 64 keys of a contiguous cache),
+// each group holding its NDB 64-column blocks of 2^lp rows of 128 bytes: one TMA box per group
+// fills it. The 128-byte swizzle moves 16-byte chunk c of a row to c ^ (key & 7).
+template <int NDB, bool kPaged>
+__device__ __forceinline__ uint32_t dec_swz(int key, int d, int lp) {
+  if constexpr (!kPaged)  // one group of 64 keys: key < 64
+    return static_cast<uint32_t>((d >> 6) * (64 * 128) + key * 128 +
+                                 ((((d & 63) >> 3) ^ (key & 7)) << 4));
+  const int grp = key >> lp, kin = key & ((1 << lp) - 1);
+  return static_cast<uint32_t>(((((grp * NDB + (d >> 6)) << lp) + kin) << 7) +
                                ((((d & 63) >> 3) ^ (key & 7)) << 4));
 }
 
@@ -99,7 +107,9 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <int D>
+// kPaged: the cache is a paged pool (p.page > 0); the contiguous instance keeps the tile layout's
+// key groups at their compile-time size of 64.
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(160)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
@@ -202,11 +212,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
             int blk = p.block_table[static_cast<long long>(b) * p.max_blocks + rr / p.page];
             if (blk < 0 || blk >= p.num_blocks) blk = p.num_blocks;  // past the map: zeros
             const int z = blk * p.Hkv + g;
-            const uint32_t o = static_cast<uint32_t>((r0 - key0) * 128);
-#pragma unroll
-            for (int db = 0; db < C::NDB; ++db) {
-              tma_load_3d(dst + db * C::BOX + o, &tm_k, db * 64, 0, z, full(st));
-              tma_load_3d(dst + C::TILE + db * C::BOX + o, &tm_v, db * 64, 0, z, full(st));
+            // the page's group: its column blocks one after the other (one box)
+            const uint32_t o = static_cast<uint32_t>((r0 - key0) * 128 * C::NDB);
+            if constexpr (C::NDB == 2) {
+              tma_load_4d(dst + o, &tm_k, 0, 0, 0, z, full(st));
+              tma_load_4d(dst + C::TILE + o, &tm_v, 0, 0, 0, z, full(st));
+            } else {
+              tma_load_3d(dst + o, &tm_k, 0, 0, z, full(st));
+              tma_load_3d(dst + C::TILE + o, &tm_v, 0, 0, z, full(st));
             }
           }
         }
@@ -260,6 +273,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   const float sl2 = p.scale_log2;
   const int mi = lane >> 3, rr = lane & 7;
   const int krow = cw * 16;
+  const int lp = kPaged ? __ffs(p.page) - 1 : 6;  // log2 of the keys per TMA group
 
   bool ok = true;
   for (int t = 0; t < n_tiles; ++t) {
@@ -277,7 +291,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
       for (int idx = lane; idx < 16 * (D / 8); idx += 32) {
         const int i = idx / (D / 8), c8 = idx % (D / 8);
         const int kk = tile0 + krow + i;
-        if (kk < klo || kk >= kend) st_shared_zero16(vS + dec_swz(krow + i, 8 * c8));
+        if (kk < klo || kk >= kend) st_shared_zero16(vS + dec_swz<C::NDB, kPaged>(krow + i, 8 * c8, lp));
       }
       __syncwarp();
     }
@@ -287,7 +301,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(kS + dec_swz(krow + (mi & 1) * 8 + rr, 16 * ks + (mi >> 1) * 8), a0, a1, a2, a3);
+      ldsm_x4(kS + dec_swz<C::NDB, kPaged>(krow + (mi & 1) * 8 + rr, 16 * ks + (mi >> 1) * 8, lp), a0, a1,
+              a2, a3);
       mma_bf16_16816(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
     }
     // sc[0]/[1]: key krow+r, heads 2c/2c+1; sc[2]/[3]: key krow+r+8
@@ -324,7 +339,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
       uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(vS + dec_swz(krow + (mi >> 1) * 8 + rr, 16 * mt + (mi & 1) * 8), a0, a1, a2, a3);
+      ldsm_x4_t(vS + dec_swz<C::NDB, kPaged>(krow + (mi >> 1) * 8 + rr, 16 * mt + (mi & 1) * 8, lp), a0,
+                a1, a2, a3);
       mma_bf16_16816(acc[mt], a0, a1, a2, a3, b0, b1);
     }
     if (edge) fence_proxy_async_smem();  // the generic zeroing before the next TMA fill

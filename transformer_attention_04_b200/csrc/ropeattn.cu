@@ -117,8 +117,10 @@ ra_status device_state(DeviceState** out) {
       st.status = static_cast<unsigned int*>(p);
       if ((e = set_smem(ra::attn_fwd_sm100_kernel<64>, ra::FwdCfg<64>::SMEM)) != cudaSuccess ||
           (e = set_smem(ra::attn_fwd_sm100_kernel<128>, ra::FwdCfg<128>::SMEM)) != cudaSuccess ||
-          (e = set_smem(ra::decode_split_kernel<64>, ra::DecCfg<64>::SMEM)) != cudaSuccess ||
-          (e = set_smem(ra::decode_split_kernel<128>, ra::DecCfg<128>::SMEM)) != cudaSuccess)
+          (e = set_smem(ra::decode_split_kernel<64, false>, ra::DecCfg<64>::SMEM)) != cudaSuccess ||
+          (e = set_smem(ra::decode_split_kernel<128, false>, ra::DecCfg<128>::SMEM)) != cudaSuccess ||
+          (e = set_smem(ra::decode_split_kernel<64, true>, ra::DecCfg<64>::SMEM)) != cudaSuccess ||
+          (e = set_smem(ra::decode_split_kernel<128, true>, ra::DecCfg<128>::SMEM)) != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute");
     }
     if (st.sm100) {
@@ -184,6 +186,36 @@ ra_status make_map(CUtensorMap* m, const void* ptr, int D, int S, long long BH, 
   if (r != CUDA_SUCCESS) {
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
                   "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return RA_ERR_CUDA;
+  }
+  return RA_OK;
+}
+
+// Paged-pool maps at D = 128: dimensions (64 columns, rows, 2 column blocks, slices) with the
+// column blocks 128 bytes apart, so that one box of (64, page, 2) brings a whole page: its two
+// 128-byte swizzled column blocks one after the other. Half the TMA operations of two
+// (64, page) boxes; the scattered 4 KB page reads are bound by that count.
+ra_status make_map_dec(CUtensorMap* m, const void* ptr, int D, int S, long long BH, int box_rows,
+                       long long rows_alloc = 0) {
+  if (D != 128) return make_map(m, ptr, D, S, BH, box_rows, rows_alloc);
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "cuTensorMapEncodeTiled entry point not found");
+    return RA_ERR_CUDA;
+  }
+  if (rows_alloc <= 0) rows_alloc = S;
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(S), 2, static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, 128,
+                                 static_cast<cuuint64_t>(rows_alloc) * D * 2};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 2, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "cuTensorMapEncodeTiled (decode, 4-D) failed (CUresult %d)", static_cast<int>(r));
     return RA_ERR_CUDA;
   }
   return RA_OK;
@@ -763,8 +795,8 @@ ra_status decode_impl(const DecodeArgs& a, cudaStream_t s) {
   CUtensorMap tk, tv;
   if (paged) {
     const long long rows = static_cast<long long>(a.num_blocks) * Hkv;
-    rs = make_map(&tk, a.k_cache, D, a.page, rows, a.page);
-    if (rs == RA_OK) rs = make_map(&tv, a.v_cache, D, a.page, rows, a.page);
+    rs = make_map_dec(&tk, a.k_cache, D, a.page, rows, a.page);
+    if (rs == RA_OK) rs = make_map_dec(&tv, a.v_cache, D, a.page, rows, a.page);
   } else {
     const long long bkv = static_cast<long long>(B) * Hkv;
     rs = make_map(&tk, a.k_cache, D, a.S_cache, bkv, 64);
@@ -805,10 +837,14 @@ ra_status decode_impl(const DecodeArgs& a, cudaStream_t s) {
   p.S_cache = a.S_cache;
   const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(B * Hkv * hblocks));
   const int pi = prof_start(1, s);
-  if (D == 64)
-    ra::decode_split_kernel<64><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
+  if (D == 64 && paged)
+    ra::decode_split_kernel<64, true><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
+  else if (D == 64)
+    ra::decode_split_kernel<64, false><<<grid, 160, ra::DecCfg<64>::SMEM, s>>>(tk, tv, p);
+  else if (paged)
+    ra::decode_split_kernel<128, true><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
   else
-    ra::decode_split_kernel<128><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
+    ra::decode_split_kernel<128, false><<<grid, 160, ra::DecCfg<128>::SMEM, s>>>(tk, tv, p);
   prof_stop(1, pi, s);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) {
