@@ -320,7 +320,9 @@ def run_ours(args):
     op = torch.empty_like(g_qp)
     od = torch.empty_like(g_qd)
     W = PREFILL_W
-    launches_per_step = 5  # table, K rotation, attention | decode split, combine
+    # K rotation, attention | decode split, combine (the cos/sin table is built at the first
+    # call and kept, so no table launch falls inside the timed region)
+    launches_per_step = 4
 
     def step(evs=None):
         if evs:
@@ -353,9 +355,15 @@ def run_ours(args):
     ra.rope_attn_profile_enable(True)
     barrier(world)
     torch.cuda.synchronize()
+    # the library's kernel events sit between a call's kernels, where they hold back the
+    # programmatic overlap of each kernel's start with the previous one's end: odd steps carry
+    # them (the kernel rooflines), even steps run as a user's calls do (the call figures)
+    K = args.steps
+    profiled = [K == 1 or i % 2 == 1 for i in range(K)]
     t_start.record()
     host_s = []
-    for i in range(args.steps):
+    for i in range(K):
+        ra.rope_attn_profile_pause(not profiled[i])
         h0 = time.perf_counter()
         step(evs[i])
         host_s.append(time.perf_counter() - h0)
@@ -370,14 +378,19 @@ def run_ours(args):
         raise RuntimeError("device timeout in the timed region")
 
     total_ms = t_start.elapsed_time(t_end)
-    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    plain = [e for e, pr in zip(evs, profiled) if not pr]
+    timing = (f"value and the call figures: the {len(plain)} timed steps without kernel events; "
+              f"roofline: the library's kernel events of the other {K - len(plain)}"
+              if plain else "one timed step: calls timed with the kernel events inside")
+    plain = plain or evs
+    n_calls = len(plain)
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in plain)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in plain)
     total_ms, pre_ms, dec_ms, k_ms, d_ms = max_over_ranks([total_ms, pre_ms, dec_ms, k_ms, d_ms],
                                                           world, dev)
-    K = args.steps
     peaks, peak_src = measured_peaks()
-    value = world * W.flops() * K / (pre_ms * 1e-3) / 1e12
-    dec_gbs = world * DECODE_W.io_bytes() * K / (dec_ms * 1e-3) / 1e9
+    value = world * W.flops() * n_calls / (pre_ms * 1e-3) / 1e12
+    dec_gbs = world * DECODE_W.io_bytes() * n_calls / (dec_ms * 1e-3) / 1e9
     attn_tflops = W.flops() / (k_ms / k_n * 1e-3) / 1e12
     split_gbs = DECODE_W.io_bytes() / (d_ms / d_n * 1e-3) / 1e9
 
@@ -387,7 +400,7 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_block(world),
         "frac_spec_bf16": value / world / SPEC_BF16_TFLOPS,
-        "decode": {"value": dec_gbs, "unit": "GB/s", "us_per_call": 1e3 * dec_ms / K,
+        "decode": {"value": dec_gbs, "unit": "GB/s", "us_per_call": 1e3 * dec_ms / n_calls,
                    "frac_spec_hbm": dec_gbs / world / SPEC_HBM_GBS,
                    "splits": ra.rope_attn_decode_auto_splits(DECODE_W.B, DECODE_W.Hq, DECODE_W.Hkv,
                                                              DECODE_W.Sk, DECODE_W.D,
@@ -397,7 +410,8 @@ def run_ours(args):
                                 "peak_source": peak_src,
                                 "kernel": "decode_split_kernel<128, false>",
                                 "traffic": recorded_traffic("decode_split_kernel decode")}},
-        "prefill_ms_per_call": pre_ms / K,
+        "prefill_ms_per_call": pre_ms / n_calls,
+        "call_timing": timing,
         # the host's own cost per step: the median over the first steps, which run before
         # the launch queue fills (later enqueues wait for the GPU to free queue space)
         "host_us_per_step": 1e6 * statistics.median(host_s[:20]),

@@ -301,8 +301,16 @@ RA_API long long rope_attn_set_wait_limit(long long limit);
  * first 1024 launches of each kind (so that profiled calls only record events; more are made
  * as needed) and returns RA_ERR_CUDA if that fails. Meant for one device at a time; not for
  * concurrent callers.
+ *
+ * rope_attn_profile_pause(1) stops the recording without ending the session: calls made
+ * while paused record nothing and run exactly as they do with profiling off (the event pairs
+ * sit between a call's kernels, where they hold back the programmatic overlap of one
+ * kernel's start with the previous kernel's end). rope_attn_profile_pause(0) resumes; the
+ * pairs recorded before the pause are kept for rope_attn_profile_read. Returns
+ * RA_ERR_INVALID_ARG when profiling is not enabled. Enabling clears the pause.
  */
 RA_API ra_status rope_attn_profile_enable(int enable);
+RA_API ra_status rope_attn_profile_pause(int pause);
 RA_API ra_status rope_attn_profile_read(int which, double* total_ms, int* launches);
 
 /* Text of a status code; the last CUDA error string for RA_ERR_CUDA. */

@@ -279,3 +279,10 @@ def test_view_rows_of_real_layouts():
     assert view_rows(tuple(cols.shape), cols.stride()) is None
     heads = x[:, :2]                                                          # uneven batch step
     assert view_rows(tuple(heads.shape), heads.stride()) is None
+
+
+def test_profile_pause_needs_a_session(lib):
+    # disabling needs no device; a pause outside a session is refused
+    assert lib.rope_attn_profile_enable(0) == ra.RA_OK
+    assert lib.rope_attn_profile_pause(1) == ra.RA_ERR_INVALID_ARG
+    assert lib.rope_attn_profile_pause(0) == ra.RA_ERR_INVALID_ARG

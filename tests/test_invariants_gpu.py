@@ -105,3 +105,27 @@ def test_wait_timeout_reports_and_recovers():
     again = ra.rope_attn_fwd(q, k, v, 500000.0)
     assert ra.rope_attn_get_device_status() == ra.RA_OK
     assert torch.equal(again, good)
+
+
+def test_profile_pause_records_nothing():
+    # a paused session records no kernel events, keeps what it had and resumes counting;
+    # the paused call's output equals the profiled one
+    q, k, v = rnd(1, 4, 300, 128, seed=40), rnd(1, 2, 300, 128, seed=41), rnd(1, 2, 300, 128, seed=42)
+    qd, kd, vd = rnd(2, 8, 1, 128, seed=43), rnd(2, 2, 512, 128, seed=44), rnd(2, 2, 512, 128, seed=45)
+    ra.rope_attn_profile_enable(True)
+    try:
+        o1 = ra.rope_attn_fwd(q, k, v, 10000.0)
+        d1 = ra.rope_attn_decode(qd, kd, vd, 10000.0, 511)
+        ra.rope_attn_profile_pause(True)
+        o2 = ra.rope_attn_fwd(q, k, v, 10000.0)
+        d2 = ra.rope_attn_decode(qd, kd, vd, 10000.0, 511)
+        ra.rope_attn_profile_pause(False)
+        o3 = ra.rope_attn_fwd(q, k, v, 10000.0)
+        torch.cuda.synchronize()
+        ms0, n0 = ra.rope_attn_profile_read(0)
+        ms1, n1 = ra.rope_attn_profile_read(1)
+    finally:
+        ra.rope_attn_profile_enable(False)
+    assert (n0, n1) == (2, 1)
+    assert ms0 > 0 and ms1 > 0
+    assert torch.equal(o1, o2) and torch.equal(o1, o3) and torch.equal(d1, d2)

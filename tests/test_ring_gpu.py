@@ -302,6 +302,18 @@ def test_partial_two_query_segments():
     _check_lse(lse, want_l, "two segments")
 
 
+def test_rotate_in_place():
+    # 5 heads: one full group of four heads per work item and a ragged group of one
+    x = _bf16((1, 5, 333, 128), 29)
+    xg = x.cuda()
+    y = ra.rope_attn_rotate(xg, 500000.0, 77)
+    ra.rope_attn_rotate(xg, 500000.0, 77, out=xg)
+    _ok()
+    assert torch.equal(xg, y)
+    want = oracle.rope_rotate(to_f64(x), 77 + np.arange(333), 500000.0)
+    assert np.max(np.abs(y.double().cpu().numpy() - want)) <= 2 ** -7 * max(1.0, np.max(np.abs(want)))
+
+
 def test_rotate_views():
     # rotate rows [30, 130) of one tensor into rows [10, 110) of another at positions 500..
     x = _bf16((2, 3, 160, 64), 28)

@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     rope_attn_get_device_status,
     rope_attn_prefill,
     rope_attn_profile_enable,
+    rope_attn_profile_pause,
     rope_attn_profile_read,
     rope_attn_rotate,
     rope_attn_set_wait_limit,

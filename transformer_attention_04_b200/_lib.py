@@ -40,6 +40,7 @@ SIGNATURES = {
     "rope_attn_last_cuda_error": (ctypes.c_char_p, []),
     "rope_attn_version": (_I, []),
     "rope_attn_profile_enable": (_I, [_I]),
+    "rope_attn_profile_pause": (_I, [_I]),
     "rope_attn_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I)]),
 }
 
@@ -365,6 +366,11 @@ def rope_attn_version() -> int:
 
 def rope_attn_profile_enable(enable: bool = True) -> None:
     _raise(lib().rope_attn_profile_enable(int(bool(enable))), "rope_attn_profile_enable")
+
+
+def rope_attn_profile_pause(pause: bool = True) -> None:
+    """Stop (or resume) recording kernel events without ending the profiling session."""
+    _raise(lib().rope_attn_profile_pause(int(bool(pause))), "rope_attn_profile_pause")
 
 
 def rope_attn_profile_read(which: int):

@@ -243,10 +243,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // launched behind the key rotation with a programmatic dependency: the set-up above overlaps
-  // its tail, the rotated keys and the table are read only after it has completed. A chained
-  // ring block (dep_late) reads only inputs that were complete before that kernel started and
-  // waits before its first merge instead. Either way the next launch may start its set-up.
+  // Only a chained ring block (dep_late) is launched with a programmatic dependency on the
+  // kernel before it (the previous block): it reads only inputs that were complete before that
+  // kernel started and waits before its first merge. Other launches are plain, where this wait
+  // returns at once. Either way the next launch, a chained block, may start its set-up.
   if (!p.dep_late) grid_dep_wait();
   grid_dep_launch();
 

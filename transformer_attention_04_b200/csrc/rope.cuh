@@ -54,43 +54,65 @@ __device__ __forceinline__ uint4 rotate8(uint4 x, const float2 (&cs)[4]) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// x, y: [nrows_total = BH * S, D] bf16, row r at sequence index r % S.
+// Heads per work item of the two elementwise kernels below: an item is one (position, 16-byte
+// chunk) of kRotHeads heads, so its angles are read (or formed) once and its kRotHeads loads
+// are in flight together before the first store.
+constexpr int kRotHeads = 4;
+
+// Work items of rope_rotate_kernel / cache_write_kernel over `heads` heads of S rows.
+__host__ __device__ inline long long rope_items(long long heads, int S, int D) {
+  return (heads + kRotHeads - 1) / kRotHeads * S * (D / 8);
+}
+
+// (cos, sin) of the 4 pairs of 16-byte chunk `chunk` at table row `row`.
+__device__ __forceinline__ void table_cs(const float2* __restrict__ tab, long long row, int chunk,
+                                         int D, float2 (&cs)[4]) {
+  const float4* t4 = reinterpret_cast<const float4*>(tab + row * (D / 2) + chunk * 4);
+  const float4 a = __ldg(t4), b = __ldg(t4 + 1);
+  cs[0] = make_float2(a.x, a.y);
+  cs[1] = make_float2(a.z, a.w);
+  cs[2] = make_float2(b.x, b.y);
+  cs[3] = make_float2(b.z, b.w);
+}
+
+// x, y: `heads` = nrows_total / S heads of S rows of D bf16; row s of head h at h * x_rows + s
+// (x) and h * y_rows + s (y); rows sit at sequence index s.
 // kTable: angles from `tab` (row tab_off + s); else computed here at pos0 + s.
+// In place (x == y, x_rows == y_rows) is allowed: each thread reads its chunks before it
+// writes them.
 template <bool kTable>
-__global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* __restrict__ x,
-                                                          uint4* __restrict__ y,
+__global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* x, uint4* y,
                                                           const float2* __restrict__ tab,
                                                           long long nrows_total, int S, int D,
                                                           long long pos0, int tab_off,
                                                           float base, int x_rows, int y_rows) {
-  // the attention kernel launched next may start its set-up now (it waits for this grid)
-  grid_dep_launch();
-  // x_rows / y_rows: rows between consecutive heads of x and y (S when packed)
   const int cpr = D / 8;  // 16-byte chunks per row
-  const long long n = nrows_total * cpr;
+  const long long heads = nrows_total / S;
+  const long long per_group = static_cast<long long>(S) * cpr;
+  const long long n = rope_items(heads, S, D);
   const double log2_base = kTable ? 0.0 : log2(static_cast<double>(base));
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
-    const long long row = e / cpr;
-    const int chunk = static_cast<int>(e - row * cpr);
-    const long long bh = row / S;
-    const int s = static_cast<int>(row - bh * S);
-    const long long xi = (bh * x_rows + s) * cpr + chunk, yi = (bh * y_rows + s) * cpr + chunk;
-    const uint4 v = __ldg(x + xi);
+    const long long grp = e / per_group;
+    const long long rem = e - grp * per_group;
+    const int s = static_cast<int>(rem / cpr);
+    const int chunk = static_cast<int>(rem - static_cast<long long>(s) * cpr);
+    const long long h0 = grp * kRotHeads;
+    const int nh = heads - h0 < kRotHeads ? static_cast<int>(heads - h0) : kRotHeads;
+    uint4 v[kRotHeads];
+#pragma unroll
+    for (int h = 0; h < kRotHeads; ++h)
+      if (h < nh) v[h] = x[((h0 + h) * x_rows + s) * cpr + chunk];
     float2 cs[4];
     if (kTable) {
-      const float4* t4 =
-          reinterpret_cast<const float4*>(tab + static_cast<long long>(tab_off + s) * (D / 2) + chunk * 4);
-      const float4 a = __ldg(t4), b = __ldg(t4 + 1);
-      cs[0] = make_float2(a.x, a.y);
-      cs[1] = make_float2(a.z, a.w);
-      cs[2] = make_float2(b.x, b.y);
-      cs[3] = make_float2(b.z, b.w);
+      table_cs(tab, tab_off + s, chunk, D, cs);
     } else {
 #pragma unroll
       for (int t = 0; t < 4; ++t) rope_cos_sin(pos0 + s, chunk * 4 + t, D, log2_base, cs[t].x, cs[t].y);
     }
-    y[yi] = rotate8(v, cs);
+#pragma unroll
+    for (int h = 0; h < kRotHeads; ++h)
+      if (h < nh) y[((h0 + h) * y_rows + s) * cpr + chunk] = rotate8(v[h], cs);
   }
 }
 
@@ -104,23 +126,36 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restric
                                                           const float2* __restrict__ tab,
                                                           long long bh_count, int S, int S_cache,
                                                           int pos0, int D, int tab_off) {
-  grid_dep_launch();  // as in rope_rotate_kernel
   const int cpr = D / 8;
-  const long long n = bh_count * S * cpr;
+  const long long per_group = static_cast<long long>(S) * cpr;
+  const long long n = rope_items(bh_count, S, D);
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
-    const long long row = e / cpr;
-    const int chunk = static_cast<int>(e - row * cpr);
-    const long long bh = row / S;
-    const int s = static_cast<int>(row - bh * S);
-    const long long dst = (bh * S_cache + pos0 + s) * cpr + chunk;
-    const float4* t4 =
-        reinterpret_cast<const float4*>(tab + static_cast<long long>(tab_off + s) * (D / 2) + chunk * 4);
-    const float4 a = __ldg(t4), b = __ldg(t4 + 1);
-    const float2 cs[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y),
-                          make_float2(b.z, b.w)};
-    kc[dst] = rotate8(__ldg(k + e), cs);
-    vc[dst] = __ldg(v + e);
+    const long long grp = e / per_group;
+    const long long rem = e - grp * per_group;
+    const int s = static_cast<int>(rem / cpr);
+    const int chunk = static_cast<int>(rem - static_cast<long long>(s) * cpr);
+    const long long h0 = grp * kRotHeads;
+    const int nh = bh_count - h0 < kRotHeads ? static_cast<int>(bh_count - h0) : kRotHeads;
+    uint4 kv[kRotHeads], vv[kRotHeads];
+#pragma unroll
+    for (int h = 0; h < kRotHeads; ++h) {
+      if (h < nh) {
+        const long long src = ((h0 + h) * S + s) * cpr + chunk;
+        kv[h] = __ldg(k + src);
+        vv[h] = __ldg(v + src);
+      }
+    }
+    float2 cs[4];
+    table_cs(tab, tab_off + s, chunk, D, cs);
+#pragma unroll
+    for (int h = 0; h < kRotHeads; ++h) {
+      if (h < nh) {
+        const long long dst = ((h0 + h) * S_cache + pos0 + s) * cpr + chunk;
+        kc[dst] = rotate8(kv[h], cs);
+        vc[dst] = vv[h];
+      }
+    }
   }
 }
 
