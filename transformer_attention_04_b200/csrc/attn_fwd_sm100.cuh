@@ -219,7 +219,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(C::B_SFULL + i), 1);
       mbar_init(bar(C::B_PFULL + i), 4);   // one arrival per softmax warp
       mbar_init(bar(C::B_OFULL + i), 1);
-      mbar_init(bar(C::B_QSTAGED + i), ns);  // one TMA store per slot
+      // one TMA store per slot, or (partial mode) one arrival per softmax warp
+      mbar_init(bar(C::B_QSTAGED + i), p.o_acc != nullptr ? 4 * ns : ns);
       mbar_init(bar(C::B_EPI + i), 4);
     }
     mbar_init(bar(C::B_DRAIN), 1);
@@ -273,8 +274,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (k >= 2 && !mbar_wait(bar(C::B_QEMPTY + qb), ((k - 2) >> 1) & 1, lim, abort_flag,
                                  p.status))
           return false;
-        // (plain mode) unit k - 2's outputs were staged in this buffer: their store has read it
-        if (k >= 2 && p.o_acc == nullptr &&
+        // unit k - 2's outputs were staged in this buffer: it has been read out
+        if (k >= 2 &&
             !mbar_wait(bar(C::B_QSTAGED + qb), ((k - 2) >> 1) & 1, lim, abort_flag, p.status))
           return false;
         const Unit w = unit_at(p, u);
@@ -300,13 +301,34 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         ++i;
         return true;
       };
+      // (partial mode, merging) the accumulator rows the unit's epilogue reads, brought into
+      // L2 a few tiles ahead so that its loads do not wait on DRAM
+      auto prefetch_acc = [&](const Unit& w) {
+        for (int s = 0; s < ns; ++s) {
+          const int q0s = w.q0 + slot_dq(p, s);
+          const int nrows = min(128, p.Sq - q0s);
+          if (nrows <= 0) continue;
+          const long long row0 =
+              static_cast<long long>(w.b * p.Hq + w.h0 + slot_dh(p, s)) * p.acc_rows + q0s;
+          bulk_prefetch_l2(p.o_acc + row0 * D, static_cast<uint32_t>(nrows * D * 4));
+          // the rows' LSE: every 128-byte line of [row0, row0 + nrows)
+          for (int j = 0; j < nrows; j += 32) prefetch_l2_line(p.lse_acc + row0 + j);
+          prefetch_l2_line(p.lse_acc + row0 + nrows - 1);
+        }
+      };
+      const bool merging = p.o_acc != nullptr && p.accumulate;
       ok = load_q(0);
       for (int k = 0; ok && unit_of(p, k) >= 0; ++k) {
         const Unit w = unit_at(p, unit_of(p, k));
+        const int jp = max(0, w.n_it - 3);  // the tile whose loads carry the prefetch
         // this unit's first K/V tile, then the next unit's Q (its buffer frees once the
         // unit before this one has issued its last S), then the rest of this unit's tiles
         ok = load_kv(w, 0, 0) && load_kv(w, 0, 1) && load_q(k + 1);
-        for (int jj = 1; ok && jj < w.n_it; ++jj) ok = load_kv(w, jj, 0) && load_kv(w, jj, 1);
+        if (ok && merging && jp == 0) prefetch_acc(w);
+        for (int jj = 1; ok && jj < w.n_it; ++jj) {
+          ok = load_kv(w, jj, 0) && load_kv(w, jj, 1);
+          if (ok && merging && jj == jp) prefetch_acc(w);
+        }
       }
       if (*abort_flag) {
         // let every copy this thread started land before the CTA can exit
@@ -631,11 +653,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!ok) break;
       // ---- epilogue of the unit: once its last PV_s has completed, O_s is read out of TMEM
       // before this warpgroup's next P (and so before the next unit's first PV_s) exists
-      if (!mbar_wait_warp(bar(C::B_OFULL + s), k & 1, lim, abort_flag, p.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      auto wait_o = [&]() -> bool {
+        if (!mbar_wait_warp(bar(C::B_OFULL + s), k & 1, lim, abort_flag, p.status)) return false;
+        tc_fence_after();
+        return true;
+      };
       if (p.o_acc != nullptr) {
         if (p.dep_late) grid_dep_wait();  // the previous kernel's merges are complete
         // partial mode: O / l and the LSE in fp32, merged with the running result
@@ -654,43 +676,108 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             lse_out = mx + logf(den);
           }
         }
-        float4* acc = reinterpret_cast<float4*>(p.o_acc + row * D);
-        __nv_bfloat16* orow = p.out ? p.out + row * D : nullptr;
+        // The warp moves its 32 rows through its quarter of the slot's Q tile (no MMA reads it
+        // any more: the unit's last S_s completed before its last P), CW columns at a time, so
+        // that global loads and stores cover whole row segments: in a coalesced pass lane l
+        // takes 16-byte chunk l % CPR of row l / CPR + RPI * i; in the row pass each thread
+        // merges its own row. Chunk ch of row rr sits at rr * 4CW + 16 (ch ^ (rr & 7)) in the
+        // stage. The first columns' old values are staged while the unit's last PV runs.
+        constexpr int CW = D / 2;        // columns per pass: 32 rows x CW fp32 = a quarter tile
+        constexpr int CPR = CW / 4;      // 16-byte fp32 chunks per row segment
+        constexpr int RPI = 32 / CPR;    // rows per coalesced instruction
+        constexpr int LPR = CW / 8;      // lanes per row segment of the bf16 copy
+        const int qb = k & 1;
+        uint8_t* stg = smem + C::OFF_Q + (qb * 2 + s) * C::TILE + qd * (32 * CW * 4);
+        const long long wrow0 =
+            static_cast<long long>(w.b * p.Hq + head) * p.acc_rows + q0s + qd * 32;
+        const int wrows = min(32, p.Sq - (q0s + qd * 32));  // this warp's rows that exist
+        const bool any_old = __any_sync(0xffffffffu, w_old != 0.f);
+        auto sw = [](int rr, int ch) { return rr * (CW * 4) + ((ch ^ (rr & 7)) << 4); };
+        auto stage_old = [&](int c0) {  // the old values of the warp's rows, into the stage
+          // (some row exists here; the stage rows past the last one take copies of it)
+          const float* abase = p.o_acc + wrow0 * D + c0;
 #pragma unroll 1
-        for (int cb = 0; cb < D; cb += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + cb, o);
-          tmem_wait_ld();
-          if (qrow < p.Sq) {
-            float v[32];
+          for (int i0 = 0; i0 < CPR; i0 += 8) {
+            float4 a[8];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * w_new;
-            if (w_old != 0.f) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float4 a = acc[cb / 4 + e];
-                v[4 * e + 0] += w_old * a.x;
-                v[4 * e + 1] += w_old * a.y;
-                v[4 * e + 2] += w_old * a.z;
-                v[4 * e + 3] += w_old * a.w;
-              }
+            for (int i = 0; i < 8; ++i) {
+              const int rr = min(RPI * (i0 + i) + lane / CPR, wrows - 1), ch = lane % CPR;
+              a[i] = __ldcg(reinterpret_cast<const float4*>(abase + rr * D) + ch);
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              acc[cb / 4 + e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-            if (orow) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + cb);
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                dst[e] = make_uint4(pack_bf16(v[8 * e + 0], v[8 * e + 1]),
-                                    pack_bf16(v[8 * e + 2], v[8 * e + 3]),
-                                    pack_bf16(v[8 * e + 4], v[8 * e + 5]),
-                                    pack_bf16(v[8 * e + 6], v[8 * e + 7]));
+            for (int i = 0; i < 8; ++i) {
+              const int rr = RPI * (i0 + i) + lane / CPR, ch = lane % CPR;
+              *reinterpret_cast<float4*>(stg + sw(rr, ch)) = a[i];
             }
           }
+          __syncwarp();
+        };
+        if (any_old) stage_old(0);  // while the unit's last PV runs
+        if (!wait_o()) {
+          ok = false;
+          break;
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += CW) {
+          float* const abase = p.o_acc + wrow0 * D + c0;  // row rr of the warp: abase + rr * D
+          if (any_old && c0 > 0) stage_old(c0);
+          // this thread's row, 32 columns at a time: O / l, plus the old values, into the stage
+#pragma unroll 1
+          for (int cb = 0; cb < CW; cb += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0 + cb, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float4* sp = reinterpret_cast<float4*>(stg + sw(lane, cb / 4 + e));
+              float4 v = make_float4(__uint_as_float(o[4 * e + 0]) * w_new,
+                                     __uint_as_float(o[4 * e + 1]) * w_new,
+                                     __uint_as_float(o[4 * e + 2]) * w_new,
+                                     __uint_as_float(o[4 * e + 3]) * w_new);
+              if (w_old != 0.f) {
+                const float4 a = *sp;
+                v.x += w_old * a.x;
+                v.y += w_old * a.y;
+                v.z += w_old * a.z;
+                v.w += w_old * a.w;
+              }
+              *sp = v;
+            }
+          }
+          __syncwarp();
+          // the merged rows: fp32 into the accumulator, bf16 into out
+#pragma unroll
+          for (int i = 0; i < CPR; ++i) {
+            const int rr = RPI * i + lane / CPR, ch = lane % CPR;
+            if (rr < wrows)
+              reinterpret_cast<float4*>(abase + rr * D)[ch] =
+                  *reinterpret_cast<const float4*>(stg + sw(rr, ch));
+          }
+          if (p.out != nullptr) {
+#pragma unroll
+            for (int i = 0; i < LPR; ++i) {
+              const int rr = (32 / LPR) * i + lane / LPR, c8 = lane % LPR;
+              if (rr < wrows) {
+                const float4 x0 = *reinterpret_cast<const float4*>(stg + sw(rr, 2 * c8));
+                const float4 x1 = *reinterpret_cast<const float4*>(stg + sw(rr, 2 * c8 + 1));
+                reinterpret_cast<uint4*>(p.out + (wrow0 + rr) * D + c0)[c8] =
+                    make_uint4(pack_bf16(x0.x, x0.y), pack_bf16(x0.z, x0.w),
+                               pack_bf16(x1.x, x1.y), pack_bf16(x1.z, x1.w));
+              }
+            }
+          }
+          __syncwarp();  // the stage is reused by the next columns
         }
         if (qrow < p.Sq) p.lse_acc[row] = lse_out;
+        // this warp is done with the Q tile: the producer may reload the buffer
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_QSTAGED + qb));
       } else {
+        if (!wait_o()) {
+          ok = false;
+          break;
+        }
         // O / l -> bf16, written row by row into this slot's Q tile of the unit (no MMA reads
         // it any more: OFULL follows the unit's last S_s) in the 128-byte swizzled layout of
         // the output's tensor map; then one thread stores the tile with TMA (rows past Sq are

@@ -220,6 +220,16 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
+// Prefetch the L2 line that holds global address `a`.
+__device__ __forceinline__ void prefetch_l2_line(const void* a) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(a)) : "memory");
+}
+// Prefetch `bytes` (a multiple of 16) of global memory from a 16-byte aligned address into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(__cvta_generic_to_global(src)),
+               "r"(bytes)
+               : "memory");
+}
 // 3-D tiled load with an L2 cache policy, completing on mbarrier `bar`.
 __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int c0,
                                                  int c1, int c2, uint32_t bar, uint64_t pol) {
