@@ -131,6 +131,11 @@ def test_auto_splits_without_gpu(lib):
     s = lib.rope_attn_decode_auto_splits(32, 64, 8, 8192, 128, 8191)
     assert 1 <= s <= 128
     assert lib.rope_attn_decode_auto_splits(1, 1, 1, 10, 128, 9) == 1
+    # the contiguous cache takes the fewest splits that put two CTAs on each of 148 SMs:
+    # 256 (batch, KV head) blocks need 2; 8 blocks need 37, capped at 32
+    assert s == 2
+    assert lib.rope_attn_decode_auto_splits(1, 8, 8, 8192, 128, 8191) == 32
+    assert lib.rope_attn_decode_auto_splits(1, 8, 8, 1000, 128, 999) == 16  # keys / 64
 
 
 def test_header_is_plain_c_and_links(tmp_path, lib):

@@ -7,10 +7,11 @@ library instead of memory taken per call.
 The test calls the entry through the C ABI twice in a row, on different inputs (so a stale
 partial left by the first call would show in the second), and compares each result with the
 allocating rope_attn_decode within the parity tolerance of the other tests, and once directly
-with the fp64 oracle. It also checks that the automatic split count is lowered until the
-partials fit (the result then equals the one-split allocating decode), and that a request
-whose partials cannot fit the array, even with one split, is refused before anything is
-enqueued.
+with the fp64 oracle. It also checks that the automatic split count's partials fit the
+array for large head counts (the contiguous-cache policy takes the fewest splits that put two
+CTAs on every SM, so many heads mean one split), that the result then equals the allocating
+decode with that count, and that a request whose partials cannot fit the array, even with
+one split, is refused before anything is enqueued.
 The file is named to be collected last.
 """
 import ctypes
@@ -77,18 +78,22 @@ def test_noalloc_matches_oracle():
     assert_parity(out, oracle.rope_attn_decode(f(q), f(kc), f(vc), 500000.0, pos), "noalloc")
 
 
-def test_noalloc_lowers_the_automatic_split_count_to_fit():
-    # 21 x 800 query heads: the usual split count is 2 on a 148-SM B200, whose partials
-    # (16.7 MiB) do not fit the array; the entry lowers it to 1 split (8.3 MiB) and must
-    # then give what the allocating decode gives with one split
+def test_noalloc_automatic_split_count_fits():
+    # 21 x 800 query heads: 2100 (batch, KV head, 8-head block) CTAs already fill a 148-SM
+    # B200, so the automatic count is 1 and its partials (8.3 MiB) fit; the entry must then
+    # give what the allocating decode gives with that count. Over the shapes below, the
+    # automatic count's partials never exceed the array
     B, Hq, Hkv, Sk, D, pos = 21, 800, 10, 128, 128, 127
     auto = ra.rope_attn_decode_auto_splits(B, Hq, Hkv, Sk, D, pos)
-    if auto < 2 or _partials_bytes(B, Hq, D, auto) <= SCRATCH_BYTES:
-        pytest.skip(f"the automatic split count here is {auto}; the shape is sized for 148 SMs")
-    assert _partials_bytes(B, Hq, D, 1) <= SCRATCH_BYTES
+    assert _partials_bytes(B, Hq, D, auto) <= SCRATCH_BYTES
+    for shape in ((32, 64, 8, 8192), (1, 8, 8, 131072), (1, 64, 1, 65536), (4, 128, 128, 4096),
+                  (64, 32, 32, 2048)):
+        b, hq, hkv, sk = shape
+        a = ra.rope_attn_decode_auto_splits(b, hq, hkv, sk, D, sk - 1)
+        assert _partials_bytes(b, hq, D, a) <= SCRATCH_BYTES, (shape, a)
     for seed in (14, 15):
         q, kc, vc = _inputs(seed, B, Hq, Hkv, Sk, D)
-        ref = ra.rope_attn_decode(q, kc, vc, 500000.0, pos, n_splits=1)
+        ref = ra.rope_attn_decode(q, kc, vc, 500000.0, pos, n_splits=auto)
         st, out = _noalloc(q, kc, vc, 500000.0, pos, 0)
         assert st == ra.RA_OK, ra.lib().rope_attn_last_cuda_error()
         torch.cuda.synchronize()

@@ -236,12 +236,22 @@ int grid_for(long long work_items, int threads, int num_sms) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-int decode_splits(int B, int Hkv, int G, int L, int num_sms, int requested) {
+int decode_splits(int B, int Hkv, int G, int L, int num_sms, int requested, bool paged) {
   const int max_splits = std::max(1, (L + 63) / 64);
   if (requested > 0) return std::min(requested, max_splits);
   const long long base = static_cast<long long>(B) * Hkv * ((G + 7) / 8);
-  // Two decode CTAs fit on one SM, but one per SM already saturates HBM: waves are counted
-  // in SMs (measured on the batch-32 8k decode: 4 splits 170 us, 8 splits 174 us)
+  if (!paged) {
+    // Contiguous cache: the fewest splits that give every SM its two resident CTAs. Each more
+    // split adds a CTA ramp per slot and a partial per head (B32 Hq64 Hkv8, 8k keys, calls
+    // back to back on a B200: 1 split 164 us, 2 splits 162 us, 4 splits 168 us, 8 splits
+    // 171 us).
+    int s = 1;
+    while (s < std::min(max_splits, 32) && base * s < 2LL * num_sms) ++s;
+    return s;
+  }
+  // Paged pool: two decode CTAs fit on one SM, but one per SM already saturates HBM: waves
+  // are counted in SMs (the same decode from 16-token pages: 2 splits 163 us, 4 splits 146 us,
+  // 8 splits 152 us)
   const double slots = static_cast<double>(num_sms);
   int best = 1;
   double best_eff = -1.0;
@@ -776,7 +786,7 @@ ra_status decode_impl(const DecodeArgs& a, cudaStream_t s) {
   int chunk = 0;
   if (a.noalloc && a.n_splits > 0) {
     // an explicit split count (as clamped by the rows) must fit the scratch; checked first
-    const int req = cut(decode_splits(B, Hkv, G, span, 1, a.n_splits), &chunk);
+    const int req = cut(decode_splits(B, Hkv, G, span, 1, a.n_splits, paged), &chunk);
     if (decode_partials_bytes(B, Hq, D, req) > kDecodeScratchBytes)
       return scratch_too_small(a.who, decode_partials_bytes(B, Hq, D, req));
   }
@@ -784,7 +794,7 @@ ra_status decode_impl(const DecodeArgs& a, cudaStream_t s) {
   DeviceState* ds = nullptr;
   ra_status rs = device_state(&ds);
   if (rs != RA_OK) return rs;
-  int splits = cut(decode_splits(B, Hkv, G, span, ds->num_sms, a.n_splits), &chunk);
+  int splits = cut(decode_splits(B, Hkv, G, span, ds->num_sms, a.n_splits, paged), &chunk);
   void* scratch = nullptr;
   if (a.noalloc) {
     rs = decode_scratch(&scratch);
@@ -1054,7 +1064,7 @@ int rope_attn_decode_auto_splits(int B, int Hq, int Hkv, int Sk, int D, int pos)
   DeviceState* ds = nullptr;
   const int sms = (device_state(&ds) == RA_OK) ? ds->num_sms : 148;
   const int L = std::min(Sk, pos + 1);
-  return decode_splits(B, Hkv, Hq / Hkv, L, sms, 0);
+  return decode_splits(B, Hkv, Hq / Hkv, L, sms, 0, false);
 }
 
 ra_status rope_attn_decode(const void* q, const void* k_cache_rot, const void* v_cache,
