@@ -189,6 +189,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      // The cache is read once: its lines go first when L2 needs room, so the stream replaces
+      // its own lines rather than dirty lines that earlier kernels left (their write-back waits
+      // for a kernel with DRAM to spare)
+      const uint64_t pol = l2_policy_evict_first();
       int issued = 0;
       for (int t = 0; t < n_tiles; ++t) {
         const int st = t % C::NST;
@@ -201,8 +205,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (p.page == 0) {
 #pragma unroll
           for (int db = 0; db < C::NDB; ++db) {
-            tma_load_3d(dst + db * C::BOX, &tm_k, db * 64, key0, kv_bh, full(st));
-            tma_load_3d(dst + C::TILE + db * C::BOX, &tm_v, db * 64, key0, kv_bh, full(st));
+            tma_load_3d_hint(dst + db * C::BOX, &tm_k, db * 64, key0, kv_bh, full(st), pol);
+            tma_load_3d_hint(dst + C::TILE + db * C::BOX, &tm_v, db * 64, key0, kv_bh, full(st),
+                             pol);
           }
         } else {
           // one box per page; a page wholly outside [lo, L) loads the page of row pos_b in
@@ -215,11 +220,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
             // the page's group: its column blocks one after the other (one box)
             const uint32_t o = static_cast<uint32_t>((r0 - key0) * 128 * C::NDB);
             if constexpr (C::NDB == 2) {
-              tma_load_4d(dst + o, &tm_k, 0, 0, 0, z, full(st));
-              tma_load_4d(dst + C::TILE + o, &tm_v, 0, 0, 0, z, full(st));
+              tma_load_4d_hint(dst + o, &tm_k, 0, 0, 0, z, full(st), pol);
+              tma_load_4d_hint(dst + C::TILE + o, &tm_v, 0, 0, 0, z, full(st), pol);
             } else {
-              tma_load_3d(dst + o, &tm_k, 0, 0, z, full(st));
-              tma_load_3d(dst + C::TILE + o, &tm_v, 0, 0, z, full(st));
+              tma_load_3d_hint(dst + o, &tm_k, 0, 0, z, full(st), pol);
+              tma_load_3d_hint(dst + C::TILE + o, &tm_v, 0, 0, z, full(st), pol);
             }
           }
         }

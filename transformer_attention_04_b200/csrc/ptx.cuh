@@ -41,34 +41,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of the phase of parity `parity` (the thread is never suspended).
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Spinning form of mbar_wait for a thread on the critical path: polls with test_wait, so
-// it sees the phase complete within a few cycles instead of after a suspension. Same limit,
-// status and abort rules as mbar_wait.
-__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, long long limit,
-                                               volatile int* abort_flag, unsigned int* status) {
-  for (long long i = 0; i < limit; ++i) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-  }
-  if (limit > 0 && mbar_test_wait(bar, parity)) return true;
-  *abort_flag = 1;
-  atomicOr(status, kStatusTimeout);
-  return false;
-}
-
 // Wait for the phase of parity `parity` of barrier `bar` to complete, polling at
 // most `limit` times. On running out it records kStatusTimeout in the sticky
 // device status word, raises the CTA's abort flag and returns false; a raised
@@ -82,51 +54,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
   }
   // limit 0 gives up without looking (a wait that nothing can satisfy, for tests)
   if (limit > 0 && mbar_try_wait(bar, parity)) return true;
-  *abort_flag = 1;
-  atomicOr(status, kStatusTimeout);
-  return false;
-}
-
-// Two phases polled together: both queries are in flight at once, so a pair of barriers
-// that have already completed costs one round trip instead of two.
-__device__ __forceinline__ bool mbar_wait2(uint32_t bar1, uint32_t parity1, uint32_t bar2,
-                                           uint32_t parity2, long long limit,
-                                           volatile int* abort_flag, unsigned int* status) {
-  bool d1 = false, d2 = false;
-  for (long long i = 0; i < limit; ++i) {
-    d1 = d1 || mbar_try_wait(bar1, parity1);
-    d2 = d2 || mbar_try_wait(bar2, parity2);
-    if (d1 && d2) return true;
-    if (*abort_flag) return false;
-  }
-  if (limit > 0 && (d1 || mbar_try_wait(bar1, parity1)) && (d2 || mbar_try_wait(bar2, parity2)))
-    return true;
-  *abort_flag = 1;
-  atomicOr(status, kStatusTimeout);
-  return false;
-}
-
-// Shared-memory event counters: a cheaper signal than an mbarrier between threads of one CTA
-// (a poll is one load). The producer side adds with release semantics, the consumer loads
-// with acquire semantics; together with tcgen05.fence::before/after_thread_sync on either
-// side this orders tcgen05 operations across the two threads.
-__device__ __forceinline__ void smem_add_release(uint32_t addr, uint32_t v) {
-  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t smem_ld_acquire(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-// Wait until the counter at `addr` reaches `target` (counters only grow), with the same
-// limit, status and abort rules as mbar_wait.
-__device__ __forceinline__ bool smem_wait_count(uint32_t addr, uint32_t target, long long limit,
-                                                volatile int* abort_flag, unsigned int* status) {
-  for (long long i = 0; i < limit; ++i) {
-    if (static_cast<int>(smem_ld_acquire(addr) - target) >= 0) return true;
-    if (*abort_flag) return false;
-  }
-  if (limit > 0 && static_cast<int>(smem_ld_acquire(addr) - target) >= 0) return true;
   *abort_flag = 1;
   atomicOr(status, kStatusTimeout);
   return false;
@@ -147,22 +74,6 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, lo
     if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
   }
   const bool ok = limit > 0 && __all_sync(0xffffffffu, mbar_try_wait(bar, parity));
-  if (!ok && (threadIdx.x & 31) == 0) {
-    *abort_flag = 1;
-    atomicOr(status, kStatusTimeout);
-  }
-  __syncwarp();
-  return ok;
-}
-
-// Warp-collective spinning wait (test_wait polls; see mbar_wait_spin).
-__device__ __forceinline__ bool mbar_wait_warp_spin(uint32_t bar, uint32_t parity, long long limit,
-                                                    volatile int* abort_flag, unsigned int* status) {
-  for (long long i = 0; i < limit; ++i) {
-    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
-    if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
-  }
-  const bool ok = limit > 0 && __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
   if (!ok && (threadIdx.x & 31) == 0) {
     *abort_flag = 1;
     atomicOr(status, kStatusTimeout);
@@ -257,28 +168,15 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// 16-byte global store with an L2 cache policy.
-__device__ __forceinline__ void st_global_v4_hint(void* ptr, uint4 v, uint64_t pol) {
-  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x),
-               "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
-               : "memory");
-}
-// 3-D tiled load (coordinates innermost first) completing on mbarrier `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
-      : "memory");
-}
 
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, int c3, uint32_t bar) {
+// 4-D tiled load with an L2 cache policy, completing on mbarrier `bar`.
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap* map, int c0,
+                                                 int c1, int c2, int c3, uint32_t bar,
+                                                 uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(pol)
       : "memory");
 }
 
@@ -341,16 +239,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-// 32 lanes x 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -370,18 +258,6 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Shared-memory matrix descriptor for tcgen05.mma (sm_100 format): start address,
-// leading/stride byte offsets (all >> 4), version 1 at bit 46, layout type at bits 61-63.
-__device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr, uint32_t lbo_bytes,
-                                                   uint32_t sbo_bytes, uint32_t layout) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;
-  d |= static_cast<uint64_t>(layout & 7u) << 61;
-  return d;
-}
 constexpr uint32_t kLayoutSW128 = 2;  // 128-byte swizzle
 
 // The same descriptor split in two 32-bit words: the low word holds the start address and

@@ -57,7 +57,7 @@ __device__ __forceinline__ uint4 rotate8(uint4 x, const float2 (&cs)[4]) {
 // Heads per work item of the two elementwise kernels below: an item is one (position, 16-byte
 // chunk) of kRotHeads heads, so its angles are read (or formed) once and its kRotHeads loads
 // are in flight together before the first store.
-constexpr int kRotHeads = 4;
+constexpr int kRotHeads = 8;
 
 // Work items of rope_rotate_kernel / cache_write_kernel over `heads` heads of S rows.
 __host__ __device__ inline long long rope_items(long long heads, int S, int D) {
