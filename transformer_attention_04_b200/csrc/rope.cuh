@@ -54,14 +54,20 @@ __device__ __forceinline__ uint4 rotate8(uint4 x, const float2 (&cs)[4]) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Heads per work item of the two elementwise kernels below: an item is one (position, 16-byte
-// chunk) of kRotHeads heads, so its angles are read (or formed) once and its kRotHeads loads
-// are in flight together before the first store.
+// The two elementwise kernels below walk tiles of (kRotHeads heads) x (256 / (D/8) rows): a
+// block of 256 threads takes one tile per pass, thread t the 16-byte chunk t % (D/8) of row
+// t / (D/8) in each of the tile's heads. Each thread reads (or forms) its angles once and has
+// its kRotHeads loads in flight together before the first store. Grids are sized by
+// rope_tiles and stride over the tiles.
 constexpr int kRotHeads = 8;
+constexpr int kRotThreads = 256;
 
-// Work items of rope_rotate_kernel / cache_write_kernel over `heads` heads of S rows.
-__host__ __device__ inline long long rope_items(long long heads, int S, int D) {
-  return (heads + kRotHeads - 1) / kRotHeads * S * (D / 8);
+__host__ __device__ inline int rope_rows_per_tile(int D) { return kRotThreads / (D / 8); }
+
+// Tiles over `heads` heads of S rows.
+__host__ __device__ inline long long rope_tiles(long long heads, int S, int D) {
+  const int rpt = rope_rows_per_tile(D);
+  return (heads + kRotHeads - 1) / kRotHeads * ((S + rpt - 1) / rpt);
 }
 
 // (cos, sin) of the 4 pairs of 16-byte chunk `chunk` at table row `row`.
@@ -81,67 +87,71 @@ __device__ __forceinline__ void table_cs(const float2* __restrict__ tab, long lo
 // In place (x == y, x_rows == y_rows) is allowed: each thread reads its chunks before it
 // writes them.
 template <bool kTable>
-__global__ void __launch_bounds__(256) rope_rotate_kernel(const uint4* x, uint4* y,
-                                                          const float2* __restrict__ tab,
-                                                          long long nrows_total, int S, int D,
-                                                          long long pos0, int tab_off,
-                                                          float base, int x_rows, int y_rows) {
+__global__ void __launch_bounds__(kRotThreads) rope_rotate_kernel(const uint4* x, uint4* y,
+                                                                  const float2* __restrict__ tab,
+                                                                  long long nrows_total, int S,
+                                                                  int D, long long pos0,
+                                                                  int tab_off, float base,
+                                                                  int x_rows, int y_rows) {
   const int cpr = D / 8;  // 16-byte chunks per row
-  const long long heads = nrows_total / S;
-  const long long per_group = static_cast<long long>(S) * cpr;
-  const long long n = rope_items(heads, S, D);
+  const int rpt = rope_rows_per_tile(D);
+  const int chunk = threadIdx.x % cpr, r_in = threadIdx.x / cpr;
+  const int heads = static_cast<int>(nrows_total / S);
+  const int row_tiles = (S + rpt - 1) / rpt;
+  const int n_tiles = (heads + kRotHeads - 1) / kRotHeads * row_tiles;
   const double log2_base = kTable ? 0.0 : log2(static_cast<double>(base));
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
-       e += (long long)gridDim.x * blockDim.x) {
-    const long long grp = e / per_group;
-    const long long rem = e - grp * per_group;
-    const int s = static_cast<int>(rem / cpr);
-    const int chunk = static_cast<int>(rem - static_cast<long long>(s) * cpr);
-    const long long h0 = grp * kRotHeads;
-    const int nh = heads - h0 < kRotHeads ? static_cast<int>(heads - h0) : kRotHeads;
+  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int g = t / row_tiles;
+    const int s = (t - g * row_tiles) * rpt + r_in;
+    if (s >= S) continue;
+    const int h0 = g * kRotHeads;
+    const int nh = min(kRotHeads, heads - h0);
     uint4 v[kRotHeads];
 #pragma unroll
     for (int h = 0; h < kRotHeads; ++h)
-      if (h < nh) v[h] = x[((h0 + h) * x_rows + s) * cpr + chunk];
+      if (h < nh) v[h] = x[(static_cast<long long>(h0 + h) * x_rows + s) * cpr + chunk];
     float2 cs[4];
     if (kTable) {
       table_cs(tab, tab_off + s, chunk, D, cs);
     } else {
 #pragma unroll
-      for (int t = 0; t < 4; ++t) rope_cos_sin(pos0 + s, chunk * 4 + t, D, log2_base, cs[t].x, cs[t].y);
+      for (int t4 = 0; t4 < 4; ++t4)
+        rope_cos_sin(pos0 + s, chunk * 4 + t4, D, log2_base, cs[t4].x, cs[t4].y);
     }
 #pragma unroll
     for (int h = 0; h < kRotHeads; ++h)
-      if (h < nh) y[((h0 + h) * y_rows + s) * cpr + chunk] = rotate8(v[h], cs);
+      if (h < nh) y[(static_cast<long long>(h0 + h) * y_rows + s) * cpr + chunk] = rotate8(v[h], cs);
   }
 }
 
 // Prefill into a KV cache: the chunk's keys k [BH, S, D] are rotated (angles from table row
 // tab_off + s, i.e. position pos0 + s) into rows pos0 + s of each [S_cache, D] slice of kc,
 // and the values v are copied to the same rows of vc. One pass over the chunk.
-__global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restrict__ k,
-                                                          const uint4* __restrict__ v,
-                                                          uint4* __restrict__ kc,
-                                                          uint4* __restrict__ vc,
-                                                          const float2* __restrict__ tab,
-                                                          long long bh_count, int S, int S_cache,
-                                                          int pos0, int D, int tab_off) {
+__global__ void __launch_bounds__(kRotThreads) cache_write_kernel(const uint4* __restrict__ k,
+                                                                  const uint4* __restrict__ v,
+                                                                  uint4* __restrict__ kc,
+                                                                  uint4* __restrict__ vc,
+                                                                  const float2* __restrict__ tab,
+                                                                  long long bh_count, int S,
+                                                                  int S_cache, int pos0, int D,
+                                                                  int tab_off) {
   const int cpr = D / 8;
-  const long long per_group = static_cast<long long>(S) * cpr;
-  const long long n = rope_items(bh_count, S, D);
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
-       e += (long long)gridDim.x * blockDim.x) {
-    const long long grp = e / per_group;
-    const long long rem = e - grp * per_group;
-    const int s = static_cast<int>(rem / cpr);
-    const int chunk = static_cast<int>(rem - static_cast<long long>(s) * cpr);
-    const long long h0 = grp * kRotHeads;
-    const int nh = bh_count - h0 < kRotHeads ? static_cast<int>(bh_count - h0) : kRotHeads;
+  const int rpt = rope_rows_per_tile(D);
+  const int chunk = threadIdx.x % cpr, r_in = threadIdx.x / cpr;
+  const int heads = static_cast<int>(bh_count);
+  const int row_tiles = (S + rpt - 1) / rpt;
+  const int n_tiles = (heads + kRotHeads - 1) / kRotHeads * row_tiles;
+  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int g = t / row_tiles;
+    const int s = (t - g * row_tiles) * rpt + r_in;
+    if (s >= S) continue;
+    const int h0 = g * kRotHeads;
+    const int nh = min(kRotHeads, heads - h0);
     uint4 kv[kRotHeads], vv[kRotHeads];
 #pragma unroll
     for (int h = 0; h < kRotHeads; ++h) {
       if (h < nh) {
-        const long long src = ((h0 + h) * S + s) * cpr + chunk;
+        const long long src = (static_cast<long long>(h0 + h) * S + s) * cpr + chunk;
         kv[h] = __ldg(k + src);
         vv[h] = __ldg(v + src);
       }
@@ -151,7 +161,7 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const uint4* __restric
 #pragma unroll
     for (int h = 0; h < kRotHeads; ++h) {
       if (h < nh) {
-        const long long dst = ((h0 + h) * S_cache + pos0 + s) * cpr + chunk;
+        const long long dst = (static_cast<long long>(h0 + h) * S_cache + pos0 + s) * cpr + chunk;
         kc[dst] = rotate8(kv[h], cs);
         vc[dst] = vv[h];
       }

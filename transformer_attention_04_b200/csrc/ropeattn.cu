@@ -229,6 +229,13 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+// Blocks of the rotation kernels: one per tile (the block scheduler balances the short blocks
+// over the SMs), capped at 32 per SM for very large tensors, whose blocks then stride over
+// the remaining tiles
+int rot_grid(long long tiles, int num_sms) {
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(tiles, 32LL * num_sms)));
+}
+
 int grid_for(long long work_items, int threads, int num_sms) {
   const long long blocks = (work_items + threads - 1) / threads;
   return static_cast<int>(std::max<long long>(1, std::min<long long>(blocks, num_sms * 16LL)));
@@ -499,18 +506,17 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
                                      ds->num_sms), 256, 0, s>>>(
         const_cast<float2*>(tab), tab_pos0, tab_len, D, a.rope_base);
   const long long bkv_heads = static_cast<long long>(B) * Hkv;
-  const long long krows = bkv_heads * Sk;
   if (cached)
-    ra::cache_write_kernel<<<grid_for(ra::rope_items(bkv_heads, Sk, D), 256, ds->num_sms), 256,
-                             0, s>>>(
+    ra::cache_write_kernel<<<rot_grid(ra::rope_tiles(bkv_heads, Sk, D), ds->num_sms),
+                             ra::kRotThreads, 0, s>>>(
         static_cast<const uint4*>(a.k), static_cast<const uint4*>(a.v),
         static_cast<uint4*>(a.k_cache), static_cast<uint4*>(a.v_cache), tab,
         static_cast<long long>(B) * Hkv, Sk, a.S_cache, a.pos_offset, D, -tab_lo);
   else
-    ra::rope_rotate_kernel<true><<<grid_for(ra::rope_items(bkv_heads, Sk, D), 256, ds->num_sms),
-                                   256, 0, s>>>(
-        static_cast<const uint4*>(a.k), static_cast<uint4*>(k_rot), tab, krows, Sk, D, 0, -tab_lo,
-        a.rope_base, Sk, Sk);
+    ra::rope_rotate_kernel<true><<<rot_grid(ra::rope_tiles(bkv_heads, Sk, D), ds->num_sms),
+                                   ra::kRotThreads, 0, s>>>(
+        static_cast<const uint4*>(a.k), static_cast<uint4*>(k_rot), tab, bkv_heads * Sk, Sk, D, 0,
+        -tab_lo, a.rope_base, Sk, Sk);
 
   CUtensorMap tq, tk, tv, to;
   const long long bkv = static_cast<long long>(B) * Hkv;
@@ -1017,8 +1023,8 @@ ra_status rope_attn_rotate_rows(const void* x, void* x_rot, int B, int H, int S,
   ra_status rs = device_state(&ds);
   if (rs != RA_OK) return rs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  ra::rope_rotate_kernel<false><<<grid_for(ra::rope_items(heads, S, D), 256, ds->num_sms), 256,
-                                  0, s>>>(
+  ra::rope_rotate_kernel<false><<<rot_grid(ra::rope_tiles(heads, S, D), ds->num_sms),
+                                  ra::kRotThreads, 0, s>>>(
       static_cast<const uint4*>(x), static_cast<uint4*>(x_rot), nullptr, rows, S, D, pos_offset,
       0, rope_base, x_rows, out_rows);
   cudaError_t e = cudaGetLastError();
