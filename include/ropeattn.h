@@ -109,8 +109,10 @@ RA_API ra_status rope_attn_fwd(const void* q, const void* k, const void* v, void
  * tensor (pointer advanced by a*D elements, rows = S_alloc) and merge into the matching rows
  * of an accumulator.
  * Two query segments: with 0 < q_split < Sq, rows i >= q_split sit at q_pos1 + (i - q_split)
- * instead of q_pos0 + i (two separate slices of one sequence in one launch). Allowed only
- * with causal == 0. q_split = 0 means one segment.
+ * instead of q_pos0 + i (two separate slices of one sequence in one launch); q_pos1 >= 0 and
+ * q_pos1 + (Sq - q_split) at most 2^30. With causal, the mask uses each row's own position,
+ * q_pos1 >= k_pos0 is required too, and q_split must be a multiple of 128 (of 256 when
+ * Hq / Hkv is odd). q_split = 0 means one segment.
  * o_acc, lse_acc and out must not overlap the inputs or each other; o_acc is 16-byte
  * aligned, lse_acc 4-byte aligned. D in {64, 128}, Hq % Hkv == 0, sizes >= 1. Runs the
  * prefill kernel of rope_attn_fwd with its fp32 epilogue (one launch, plus the RoPE table of

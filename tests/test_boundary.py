@@ -248,7 +248,9 @@ def partial(lib, q=FAKE, k=FAKE + (1 << 40), v=FAKE + (2 << 40), o=FAKE + (3 << 
     (dict(q_rows=15), ra.RA_ERR_INVALID_ARG),           # head stride shorter than the rows
     (dict(kv_rows=-1), ra.RA_ERR_INVALID_ARG),
     (dict(acc_rows=8), ra.RA_ERR_INVALID_ARG),
-    (dict(split=8, qp1=100), ra.RA_ERR_INVALID_ARG),    # two query segments need causal == 0
+    (dict(split=8, qp1=100), ra.RA_ERR_INVALID_ARG),    # masked: q_split not on a 128-row edge
+    (dict(Sq=256, split=128, qp1=15, kp=16, qp=32), ra.RA_ERR_INVALID_ARG),  # 2nd segment early
+    (dict(Sq=384, Hq=6, Hkv=2, split=128, qp1=500), ra.RA_ERR_INVALID_ARG),  # odd G: 256 rows
     (dict(split=8, qp1=-1, causal=0), ra.RA_ERR_INVALID_ARG),
     (dict(split=-1), ra.RA_ERR_INVALID_ARG),
     # o_acc inside k's strided extent (2 heads 64 rows apart: 80 rows of 128 bytes)
@@ -262,6 +264,12 @@ def test_partial_noncausal_any_offsets_until_device(lib):
     # without the mask a block may sit anywhere; with no GPU the call fails at the device step
     st = partial(lib, qp=0, kp=500, causal=0)
     assert st != ra.RA_ERR_INVALID_ARG
+
+
+def test_partial_masked_two_segments_until_device(lib):
+    # a masked call with two query segments on 128-row edges passes the checks (odd G: 256)
+    for kw in (dict(Sq=256, split=128, qp1=500), dict(Sq=512, Hq=6, Hkv=2, split=256, qp1=32)):
+        assert partial(lib, **kw) != ra.RA_ERR_INVALID_ARG, kw
 
 
 def test_view_rows_of_real_layouts():

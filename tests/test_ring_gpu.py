@@ -302,6 +302,47 @@ def test_partial_two_query_segments():
     _check_lse(lse, want_l, "two segments")
 
 
+@pytest.mark.parametrize("D,G,Sq,split,Sk,d0,d1", [
+    (128, 4, 512, 256, 256, 0, 1000),  # the zig-zag step 0: a diagonal chunk, a wholly past one
+    (64, 4, 512, 256, 256, 0, 1000),
+    (128, 3, 640, 256, 300, 40, 100),  # odd group size (256-row units), both segments masked
+])
+def test_partial_two_query_segments_masked(D, G, Sq, split, Sk, d0, d1):
+    # a masked block whose two query segments sit at their own positions (rows [0, split) at
+    # kp + d0.., rows [split, Sq) at kp + d1..), merged over an earlier unmasked block of keys
+    # before kp; the mask compares each row's own position with the keys'
+    B, Hkv, base, kp = 1, 2, 500000.0, 5000
+    Hq = G * Hkv
+    q, k, v = _bf16((B, Hq, Sq, D), 34), _bf16((B, Hkv, Sk, D), 35), _bf16((B, Hkv, Sk, D), 36)
+    k0, v0 = _bf16((B, Hkv, 128, D), 37), _bf16((B, Hkv, 128, D), 38)
+    kr, kr0 = _rotated_keys(k, kp, base), _rotated_keys(k0, kp - 128, base)
+    p0, p1 = kp + d0, kp + d1
+
+    def block(qs, pos, kk, vv, kpos, causal):
+        return oracle.rope_attn_fwd_partial(to_f64(qs), to_f64(kk), to_f64(vv), base, pos, kpos,
+                                            causal)
+
+    want = []
+    for qs, pos in ((q[:, :, :split], p0), (q[:, :, split:], p1)):
+        a = block(qs, pos, kr0, v0, kp - 128, False)
+        b = block(qs, pos, kr, v, kp, True)
+        want.append(oracle.merge_partials(a[0], a[1], b[0], b[1]))
+    want_o = np.concatenate([w[0] for w in want], axis=2)
+    want_l = np.concatenate([w[1] for w in want], axis=2)
+    o_acc = torch.full((B, Hq, Sq, D), float("nan"), device="cuda")
+    lse = torch.full((B, Hq, Sq), float("nan"), device="cuda")
+    out = torch.full((B, Hq, Sq, D), float("nan"), device="cuda", dtype=torch.bfloat16)
+    qg = q.cuda()
+    ra.rope_attn_fwd_partial(qg, kr0.cuda(), v0.cuda(), o_acc, lse, base, p0, kp - 128, False,
+                             q_split=split, q_pos1=p1)
+    ra.rope_attn_fwd_partial(qg, kr.cuda(), v.cuda(), o_acc, lse, base, p0, kp, True,
+                             accumulate=True, out=out, q_split=split, q_pos1=p1)
+    _ok()
+    assert_parity(o_acc, want_o, "two masked segments")
+    assert_parity(out, want_o, "two masked segments, bf16 copy")
+    _check_lse(lse, want_l, "two masked segments")
+
+
 def test_rotate_in_place():
     # 5 heads: one full group of four heads per work item and a ragged group of one
     x = _bf16((1, 5, 333, 128), 29)

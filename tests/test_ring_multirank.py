@@ -7,6 +7,7 @@ itself: which block each rank holds at each step, which blocks it skips, the pos
 passes, the merge order and the final output. The result must equal the oracle's full
 attention over the whole sequence.
 """
+import itertools
 import os
 import socket
 import sys
@@ -54,12 +55,12 @@ def _worker(rank, world, port, causal, q_out, layout="contiguous"):
                     accumulate=False, out=None, q_split=0, q_pos1=0, chained=False):
         calls.append((q_pos0, k_pos0, bool(accumulate), out is not None))
         if 0 < q_split < q.shape[2]:
-            # two query segments (unmasked): each row's result depends only on its position
-            assert not causal
+            # two query segments: each row's result depends only on its own position (the
+            # mask, if any, compares that position with the keys')
             parts = [oracle.rope_attn_fwd_partial(q[:, :, :q_split].numpy(), k_rot.numpy(),
-                                                  v.numpy(), rope_base, q_pos0, k_pos0, False),
+                                                  v.numpy(), rope_base, q_pos0, k_pos0, causal),
                      oracle.rope_attn_fwd_partial(q[:, :, q_split:].numpy(), k_rot.numpy(),
-                                                  v.numpy(), rope_base, q_pos1, k_pos0, False)]
+                                                  v.numpy(), rope_base, q_pos1, k_pos0, causal)]
             o = np.concatenate([parts[0][0], parts[1][0]], axis=2)
             lse = np.concatenate([parts[0][1], parts[1][1]], axis=2)
         else:
@@ -170,31 +171,40 @@ def test_zigzag_ring_attention_gloo_equals_full(world, causal):
         n_calls.append(len(calls))
         # the first call of the rank overwrites, the last one writes the output
         assert not calls[0][2] and calls[-1][3]
-    # balanced: every rank makes the same launches (world + 2 masked, world unmasked)
+    # balanced: every rank makes the same launches (world unmasked; masked world + 2 here,
+    # since 3-row chunks do not fall on the kernel's 128-row unit edges)
     assert n_calls == [world + 2 if causal else world] * world
 
 
 def test_zigzag_calls_schedule():
     sys.path.insert(0, ROOT)
-    from transformer_attention_04_b200.ring import zigzag_calls
-    size = {"lo": 1, "hi": 1, "all": 2}
-    for world in (1, 2, 3, 4, 8):
+    from transformer_attention_04_b200.ring import zigzag_calls, zigzag_step0_fused
+    halves = {"lo": ["lo"], "hi": ["hi"], "all": ["lo", "hi"]}
+    for world, fused in itertools.product((1, 2, 3, 4, 8), (True, False)):
+        chunk = lambda owner, h: owner if h == "lo" else 2 * world - 1 - owner  # noqa: E731
         for r in range(world):
-            calls = zigzag_calls(r, world, True)
-            assert len(calls) == world + 2
-            # chunk blocks attended (a masked diagonal one counts half): 2*world on every rank
-            work = sum(size[qh] * size[kh] * (0.5 if m else 1) for _, _, qh, kh, m in calls)
+            calls = zigzag_calls(r, world, True, fused)
+            assert len(calls) == world + (1 if fused else 2)
+            # chunk blocks attended (a diagonal one counts half): 2*world on every rank; a
+            # masked call may hold a diagonal block and a wholly past one
+            work = sum(0.5 if chunk(r, a) == chunk(s, b) else 1
+                       for _, s, qh, kh, _ in calls for a in halves[qh] for b in halves[kh])
             assert work == 2 * world
+            # the mask is asked for exactly where a call holds a diagonal block
+            for _, s, qh, kh, m in calls:
+                assert m == any(chunk(r, a) == chunk(s, b) for a in halves[qh] for b in halves[kh])
             # every (query chunk, key chunk) pair with the key chunk not after the query chunk
             # is attended exactly once
-            chunk = lambda owner, h: owner if h == "lo" else 2 * world - 1 - owner
-            halves = {"lo": ["lo"], "hi": ["hi"], "all": ["lo", "hi"]}
             seen = sorted((chunk(r, a), chunk(s, b)) for _, s, qh, kh, _ in calls
                           for a in halves[qh] for b in halves[kh])
             want = sorted((qc, kc) for qc in (chunk(r, "lo"), chunk(r, "hi"))
                           for kc in range(2 * world) if kc <= qc)
             assert seen == want
-            assert len(zigzag_calls(r, world, False)) == world
+            assert len(zigzag_calls(r, world, False, fused)) == world
+    # the kernel's units cover 128 query rows, 256 for an odd group size
+    assert zigzag_step0_fused(256, 8, 2) and zigzag_step0_fused(2048, 64, 8)
+    assert not zigzag_step0_fused(300, 8, 2)
+    assert zigzag_step0_fused(256, 6, 2) and not zigzag_step0_fused(128, 6, 2)
 
 
 def test_ring_drivers_reject_bad_arguments():

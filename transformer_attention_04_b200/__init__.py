@@ -28,4 +28,5 @@ from ._lib import (  # noqa: F401
     rope_attn_set_wait_limit,
     rope_attn_version,
 )
-from .ring import ring_attention, ring_attention_local, ring_steps, zigzag_calls  # noqa: F401,E402
+from .ring import (ring_attention, ring_attention_local, ring_steps, zigzag_calls,  # noqa: F401,E402
+                   zigzag_step0_fused)

@@ -182,7 +182,8 @@ def rope_attn_fwd_partial(q, k_rot, v, o_acc, lse_acc, rope_base: float, q_pos0:
                           k_pos0: int, causal: bool = True, accumulate: bool = False, out=None,
                           q_split: int = 0, q_pos1: int = 0, stream=None, chained: bool = False):
     """One ring-attention block: q [B,Hq,Sq,D] (rotated here to q_pos0+i; rows >= q_split at
-    q_pos1 + (i - q_split) when 0 < q_split < Sq, unmasked calls only) against keys k_rot
+    q_pos1 + (i - q_split) when 0 < q_split < Sq: masked calls need q_split a multiple of 128,
+    of 256 for an odd group size, and q_pos1 >= k_pos0) against keys k_rot
     [B,Hkv,Sk,D] already rotated to k_pos0+j, and v. The block's normalised output and
     natural-log LSE go to o_acc [B,Hq,Sq,D] / lse_acc [B,Hq,Sq] (fp32), merged with their
     contents when ``accumulate``; ``out`` (bf16), if given, also receives the merged result.

@@ -67,6 +67,7 @@ struct FwdParams {
   int n_units;          // n_qtiles * B * Hkv * ppg
   int causal;
   int off;              // query row i sits at key index i + off (causal: key j allowed iff j <= i + off)
+  int off2;             // the same for the rows of the second query segment (i >= q_split)
   int window;           // 0 = none; else key j is allowed to query row i iff j > i + off - window
   int q_tab_off;        // query row i < q_split reads table row q_tab_off + i
   int q_split;          // first row of a second segment of positions (Sq if none)...
@@ -144,9 +145,11 @@ __device__ __forceinline__ Unit unit_at(const FwdParams& p, int u) {
   w.q0 = qg * 128 * (p.pair_q ? 2 : 1);
   const int q_last = w.q0 + slot_dq(p, p.n_slots - 1) + 127;  // the unit's last query row
   int n_kv = (p.Sk + 127) / 128;
-  if (p.causal) n_kv = min(n_kv, (min(p.Sq - 1, q_last) + p.off) / 128 + 1);
+  // a unit lies in one query segment (the host keeps q_split a multiple of its rows)
+  const int off = (w.q0 >= p.q_split) ? p.off2 : p.off;
+  if (p.causal) n_kv = min(n_kv, (min(p.Sq - 1, q_last) + off) / 128 + 1);
   // with a sliding window, tiles wholly below the first row's window are skipped too
-  w.j_lo = (p.window > 0) ? max(0, w.q0 + p.off - p.window + 1) / 128 : 0;
+  w.j_lo = (p.window > 0) ? max(0, w.q0 + off - p.window + 1) / 128 : 0;
   w.n_it = n_kv - w.j_lo;  // KV tiles visited: j_lo .. n_kv - 1
   return w;
 }
@@ -545,7 +548,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int head = w.h0 + slot_dh(p, s);
       float m = -INFINITY;  // running row max, in log2 units of the scaled score
       float l = 0.f;        // running row sum of 2^(x - m)
-      const int lim_causal = min(p.Sk - 1, qrow + p.off);
+      const int off = (q0s >= p.q_split) ? p.off2 : p.off;  // this slot's query segment
+      const int lim_causal = min(p.Sk - 1, qrow + off);
       for (int jj = 0; jj < w.n_it; ++jj, ++t) {  // KV tile j_lo + jj
         if (!mbar_wait_warp(bar(C::B_SFULL + s), t & 1, lim, abort_flag, p.status)) {
           ok = false;
@@ -562,11 +566,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         // causal / window / sequence-end mask, only on tiles that reach past some row's limit
         const int kbase = (w.j_lo + jj) * 128;
         const bool need_mask = (kbase + 128 > p.Sk) ||
-                               (p.causal && kbase + 127 > q0s + p.off) ||
-                               (p.window > 0 && kbase + p.window < q0s + 128 + p.off);
+                               (p.causal && kbase + 127 > q0s + off) ||
+                               (p.window > 0 && kbase + p.window < q0s + 128 + off);
         if (need_mask) {
           const int lim_k = (p.causal ? lim_causal : p.Sk - 1) - kbase;
-          const int lo_k = (p.window > 0) ? qrow + p.off - p.window + 1 - kbase : 0;
+          const int lo_k = (p.window > 0) ? qrow + off - p.window + 1 - kbase : 0;
           // the sign of (lim_k - c) | (c - lo_k) masks the element: integer ops, no branch or
           // predicate (the limits differ from lane to lane)
           if (p.window > 0) {

@@ -544,6 +544,7 @@ ra_status prefill_impl(const PrefillArgs& a, cudaStream_t s) {
     p.n_units = static_cast<int>(n_units);
     p.causal = a.causal ? 1 : 0;
     p.off = static_cast<int>(T) - Sq;  // bottom-right alignment of the queries on the keys
+    p.off2 = p.off;
     p.window = a.window;
     p.q_tab_off = (Sk - Sq) - tab_lo;
     p.q_split = Sq;
@@ -586,9 +587,10 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   const int kv_rows = a.kv_rows ? a.kv_rows : Sk;
   const int acc_rows = a.acc_rows ? a.acc_rows : Sq;
   if (q_rows < Sq || kv_rows < Sk || acc_rows < Sq) return RA_ERR_INVALID_ARG;
-  // a second query segment: only without the mask (the kernel's causal offset is per launch)
+  // a second query segment (rows q_split.. at q_pos1..): under the mask every row of it must
+  // see the block's first key, and q_split must fall on a work unit's edge (checked below)
   const bool two_seg = a.q_split > 0 && a.q_split < Sq;
-  if (a.q_split < 0 || (two_seg && (a.causal || a.q_pos1 < 0 ||
+  if (a.q_split < 0 || (two_seg && (a.q_pos1 < 0 || (a.causal && a.q_pos1 < a.k_pos0) ||
                                     static_cast<long long>(a.q_pos1) + (Sq - a.q_split) >
                                         (1LL << 30))))
     return RA_ERR_INVALID_ARG;
@@ -631,6 +633,9 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
   // two slots per unit: two heads of a KV group (even G) or two consecutive query tiles of
   // one head (odd G)
   const int pair_q = G % 2;
+  // each unit's rows lie in one segment: under the mask, q_split is a multiple of 128 rows
+  // (256 with two query tiles per unit)
+  if (two_seg && a.causal && a.q_split % (pair_q ? 256 : 128)) return RA_ERR_INVALID_ARG;
   const int n_qtiles = (Sq + 127) / 128;
   const int ppg = pair_q ? G : G / 2;
   const long long n_units =
@@ -682,6 +687,7 @@ ra_status partial_impl(const PartialArgs& a, cudaStream_t s) {
     p.n_units = static_cast<int>(n_units);
     p.causal = a.causal ? 1 : 0;
     p.off = a.q_pos0 - a.k_pos0;  // query row i at q_pos0 + i, key j at k_pos0 + j
+    p.off2 = two_seg ? a.q_pos1 - n0 - a.k_pos0 : p.off;  // row i >= n0 at q_pos1 + (i - n0)
     p.window = 0;
     // query row i sits at q_pos0 + i, or at q_pos1 + (i - n0) in the second segment
     p.q_tab_off = tab_cached ? a.q_pos0 : 0;

@@ -37,27 +37,39 @@ def ring_steps(rank: int, world: int, causal: bool):
     return out
 
 
-def zigzag_calls(rank: int, world: int, causal: bool):
+def zigzag_step0_fused(c: int, Hq: int, Hkv: int) -> bool:
+    """Whether step 0 can attend both query chunks in one masked launch: the kernel's work
+    units must not straddle the chunk edge (c a multiple of 128 rows, of 256 when two query
+    tiles share a unit, which an odd group size makes them do)."""
+    return c % (256 if (Hq // Hkv) % 2 else 128) == 0
+
+
+def zigzag_calls(rank: int, world: int, causal: bool, fused: bool = True):
     """The kernel calls of one rank under the zig-zag split.
 
     The sequence is cut into 2*world chunks of c tokens; rank r holds chunk r then chunk
     2*world-1-r in one [.., 2c, ..] tensor ("lo" and "hi" halves). At step t it holds the
     keys/values of rank src = (rank - t) mod world in the same layout. Returns, in order,
     (step, src, query half, key half, masked) with halves "lo", "hi" or "all":
-    * step 0: the two diagonal chunk blocks (masked) and the high query chunk against the low
-      key chunk (wholly past);
+    * step 0: both query chunks against the low key chunk in one masked launch (the low
+      chunk's diagonal block; the high chunk is wholly past it, its rows at their own
+      positions), then the high diagonal block (masked). With ``fused`` false (chunks that
+      do not fall on the kernel's unit edges, see zigzag_step0_fused) the first launch is
+      split into the low diagonal block and the wholly past high-on-low block;
     * src < rank: both query chunks against the low key chunk (wholly past: one launch, the
       two query chunks at their own positions);
     * src > rank: the high query chunk against both key chunks (wholly past: one launch);
     * blocks wholly in the future are skipped. Without the mask every step is one launch of
       all queries against all keys.
-    Every rank attends 2*world chunk blocks (counting a diagonal one as half) in world + 2
-    launches under the mask."""
+    Every rank attends 2*world chunk blocks (counting a diagonal one as half) in world + 1
+    launches under the mask (world + 2 unfused)."""
     calls = []
     for t in range(world):
         src = (rank - t) % world
         if not causal:
             calls.append((t, src, "all", "all", False))
+        elif t == 0 and fused:
+            calls += [(0, rank, "all", "lo", True), (0, rank, "hi", "hi", True)]
         elif t == 0:
             calls += [(0, rank, "lo", "lo", True), (0, rank, "hi", "lo", False),
                       (0, rank, "hi", "hi", True)]
@@ -189,7 +201,7 @@ def _ring_zigzag(q, k, v, rope_base, causal, group, out, world, rank, partial_fn
     acc_l = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     if out is None:
         out = torch.empty_like(q)
-    calls = zigzag_calls(rank, world, causal)
+    calls = zigzag_calls(rank, world, causal, zigzag_step0_fused(c, Hq, k.shape[1]))
     nxt, prv = peer((rank + 1) % world), peer((rank - 1) % world)
     i = 0
     for t in range(world):
@@ -291,7 +303,7 @@ def _ring_zigzag_local(q, k, v, rope_base, n, causal, out, on_rank):
     for r in range(n):
         if on_rank:
             on_rank(r, "start")
-        calls = zigzag_calls(r, n, causal)
+        calls = zigzag_calls(r, n, causal, zigzag_step0_fused(c, Hq, k.shape[1]))
         for i, (_, src, _, _, _) in enumerate(calls):
             # all keys were rotated before the first call (see ring_attention_local)
             _zigzag_issue(_lib.rope_attn_fwd_partial, calls, i, r, n, c, qs[r], ks[src], vs[src],
