@@ -347,8 +347,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // (S(t+1) being the S of the unit's next tile, or the next unit's first). The single
     // order makes the two slots alternate: one slot's softmax runs while the other slot's
     // MMAs execute. Each tcgen05.mma holds the issuing thread for about its duration and
-    // each barrier wait or commit costs it a few hundred cycles, so the thread keeps the
-    // code between MMAs short and waits for the ring tiles while it would wait for P anyway.
+    // each barrier wait or commit costs it a few hundred cycles even when the phase has long
+    // completed, so the thread keeps the code between MMAs short and polls the tile's V, the
+    // next K and P0 together: one round trip instead of three (the tensor pipe idles through
+    // every one of them).
     if (lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc_bf16(128, 128, 0, 0);  // Q, K both K-major
       constexpr uint32_t kIdescO = umma_idesc_bf16(128, D, 0, 1);    // V is MN-major
@@ -413,10 +415,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int qbn = last ? (k + 1) & 1 : k & 1;                  // Q buffer of the next tile
           const bool next_last = last ? n_next == 1 : jj + 2 == n_it;  // next tile ends its unit
           // the ring tiles (normally landed long ago) and the next unit's Q first, then P0
-          ok = wait(C::B_FULL + slot(2 * t + 1), par(2 * t + 1)) &&
-               (!has_next || ((!last || wait(C::B_QREADY + qbn, ((k + 1) >> 1) & 1)) &&
-                              wait(C::B_FULL + slot(2 * t + 2), par(2 * t + 2)))) &&
-               wait(C::B_PFULL + 0, t & 1);
+          // the tile's V, the next K and P0 polled together (the next unit's Q first)
+          ok = (!(has_next && last) || wait(C::B_QREADY + qbn, ((k + 1) >> 1) & 1)) &&
+               mbar_wait3(bar(C::B_PFULL + 0), t & 1, bar(C::B_FULL + slot(2 * t + 1)),
+                          par(2 * t + 1), bar(C::B_FULL + slot(2 * t + 2)), par(2 * t + 2),
+                          has_next ? 3 : 2, lim, abort_flag, p.status);
           if (!ok) break;
           // ---- slot 0: PV0(t), then S0(t + 1)
           // (P_s of a unit's first tile comes after the softmax group has read the previous

@@ -59,6 +59,29 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
   return false;
 }
 
+// Up to three phases polled together: the queries are in flight at once, so barriers that
+// have already completed cost one round trip instead of one each. n: how many of the three
+// pairs count (the rest are ignored).
+__device__ __forceinline__ bool mbar_wait3(uint32_t b1, uint32_t p1, uint32_t b2, uint32_t p2,
+                                           uint32_t b3, uint32_t p3, int n, long long limit,
+                                           volatile int* abort_flag, unsigned int* status) {
+  bool d1 = false, d2 = n < 2, d3 = n < 3;
+  for (long long i = 0; i < limit; ++i) {
+    const bool r1 = d1 || mbar_try_wait(b1, p1);
+    const bool r2 = d2 || mbar_try_wait(b2, p2);
+    const bool r3 = d3 || mbar_try_wait(b3, p3);
+    d1 = r1; d2 = r2; d3 = r3;
+    if (d1 && d2 && d3) return true;
+    if (*abort_flag) return false;
+  }
+  if (limit > 0 && (d1 || mbar_try_wait(b1, p1)) && (d2 || mbar_try_wait(b2, p2)) &&
+      (d3 || mbar_try_wait(b3, p3)))
+    return true;
+  *abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
 // Drain waits bound the exit path after an abort; they ignore the abort flag.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   for (int i = 0; i < (1 << 22); ++i)
