@@ -419,7 +419,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const bool has_next = !last || n_next > 0;
           const int qbn = last ? (k + 1) & 1 : k & 1;                  // Q buffer of the next tile
           const bool next_last = last ? n_next == 1 : jj + 2 == n_it;  // next tile ends its unit
-          // the ring tiles (normally landed long ago) and the next unit's Q first, then P0
           // the tile's V, the next K and P0 polled together (the next unit's Q first)
           ok = (!(has_next && last) || wait(C::B_QREADY + qbn, ((k + 1) >> 1) & 1)) &&
                mbar_wait3(bar(C::B_PFULL + 0), t & 1, bar(C::B_FULL + slot(2 * t + 1)),
