@@ -69,6 +69,12 @@ RAGGED = [
     (2, 4, 2, 333, 333, 128, False, 0),  # no mask
     (1, 2, 1, 200, 77, 64, False, 3),    # no mask, Sq > Sk
     (1, 4, 1, 640, 640, 128, True, 0),   # exact multiple of the tile
+    # long key ranges: 64 KV tiles per unit, so the K/V ring's slots are reused many times
+    # (D = 64 keeps K and V in separate slots of an 8-slot ring, D = 128 alternates them in 3)
+    (1, 4, 2, 256, 8192, 64, False, 0),
+    (1, 4, 2, 256, 8192, 128, False, 0),
+    (1, 3, 1, 256, 8192, 64, False, 0),  # odd group size: two query tiles per unit
+    (1, 4, 2, 2048, 2048, 64, True, 0),
 ]
 
 

@@ -293,15 +293,25 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       };
       auto load_kv = [&](const Unit& w, int jj, int kv) -> bool {  // kv 0: K, 1: V
         const int sl = i % C::NSLOT;
-        // the slot's previous item j: a V tile is released by its own commit after its last
-        // PV (EMPTY completes once per V occupant of the slot); a K tile by the last S that
-        // reads it (the SFULL commit of the tile's last slot)
-        const int j = i - C::NSLOT;
-        if (j >= 0 && !((j & 1) ? mbar_wait(bar(C::B_EMPTY + sl), ((j / C::NSLOT) >> 1) & 1, lim,
-                                            abort_flag, p.status)
-                                : mbar_wait(bar(C::B_SFULL + ns - 1), (j >> 1) & 1, lim,
-                                            abort_flag, p.status)))
-          return false;
+        const int j = i - C::NSLOT;  // the slot's previous item
+        if constexpr (C::NSLOT % 2 == 1) {
+          // K and V items alternate in each slot. A V tile is released by its own commit after
+          // its last PV (EMPTY completes once per V occupant); a K tile by the last S that reads
+          // it (the SFULL commit of the tile's last slot). K(t)'s release is checked right after
+          // K(t + 1) has been issued, and SFULL's next phase needs K(t + 1) to land: the barrier
+          // is at most one phase past the one awaited.
+          if (j >= 0 && !((j & 1) ? mbar_wait(bar(C::B_EMPTY + sl), ((j / C::NSLOT) >> 1) & 1,
+                                              lim, abort_flag, p.status)
+                                  : mbar_wait(bar(C::B_SFULL + ns - 1), (j >> 1) & 1, lim,
+                                              abort_flag, p.status)))
+            return false;
+        } else {
+          // an even ring keeps K and V in separate slots, several tiles ahead: every item is
+          // released by a commit of its own
+          if (j >= 0 && !mbar_wait(bar(C::B_EMPTY + sl), (j / C::NSLOT) & 1, lim, abort_flag,
+                                   p.status))
+            return false;
+        }
         mbar_expect_tx(bar(C::B_FULL + sl), C::TILE);
         const CUtensorMap* map = kv ? &tm_v : &tm_k;
         for (int kb = 0; kb < C::KB; ++kb)
@@ -408,6 +418,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             umma_commit(bar(C::B_SFULL + 1));
           }
           if (n_it == 1) umma_commit(bar(C::B_QEMPTY + 0));
+          if constexpr (C::NSLOT % 2 == 0) umma_commit(bar(C::B_EMPTY + slot(0)));
         }
       }
       int t = 0;
@@ -453,6 +464,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (ns == 1) umma_commit(bar(C::B_EMPTY + slot(2 * t + 1)));
           if (has_next) {
             if (next_last) umma_commit(bar(C::B_QEMPTY + qbn));  // that unit's last S
+            if constexpr (C::NSLOT % 2 == 0) umma_commit(bar(C::B_EMPTY + slot(2 * t + 2)));
           }
         }
         if (!ok || n_next == 0) break;
