@@ -355,6 +355,21 @@ def test_rotate_in_place():
     assert np.max(np.abs(y.double().cpu().numpy() - want)) <= 2 ** -7 * max(1.0, np.max(np.abs(want)))
 
 
+@pytest.mark.parametrize("D", [24, 40, 96, 120, 256])
+def test_rotate_any_row_width(D):
+    # D / 8 chunks per row: where that does not divide the rotation block, the threads past a
+    # tile's last whole row must leave the next tile's first row alone (in place it would
+    # otherwise be rotated twice)
+    x = _bf16((2, 3, 301, D), 31)
+    xg = x.cuda()
+    y = ra.rope_attn_rotate(xg, 10000.0, 5)
+    ra.rope_attn_rotate(xg, 10000.0, 5, out=xg)
+    _ok()
+    assert torch.equal(xg, y)
+    want = oracle.rope_rotate(to_f64(x), 5 + np.arange(301), 10000.0)
+    assert np.max(np.abs(y.double().cpu().numpy() - want)) <= 2 ** -7 * max(1.0, np.max(np.abs(want)))
+
+
 def test_rotate_views():
     # rotate rows [30, 130) of one tensor into rows [10, 110) of another at positions 500..
     x = _bf16((2, 3, 160, 64), 28)

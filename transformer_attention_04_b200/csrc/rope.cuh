@@ -56,9 +56,10 @@ __device__ __forceinline__ uint4 rotate8(uint4 x, const float2 (&cs)[4]) {
 
 // The two elementwise kernels below walk tiles of (kRotHeads heads) x (256 / (D/8) rows): a
 // block of 256 threads takes one tile per pass, thread t the 16-byte chunk t % (D/8) of row
-// t / (D/8) in each of the tile's heads. Each thread reads (or forms) its angles once and has
-// its kRotHeads loads in flight together before the first store. Grids are sized by
-// rope_tiles and stride over the tiles.
+// t / (D/8) in each of the tile's heads; when D/8 does not divide 256, the threads past the
+// tile's last whole row idle. Each thread reads (or forms) its angles once and has its
+// kRotHeads loads in flight together before the first store. Grids are sized by rope_tiles
+// and stride over the tiles.
 constexpr int kRotHeads = 8;
 constexpr int kRotThreads = 256;
 
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kRotThreads) rope_rotate_kernel(const uint4* x
   const int cpr = D / 8;  // 16-byte chunks per row
   const int rpt = rope_rows_per_tile(D);
   const int chunk = threadIdx.x % cpr, r_in = threadIdx.x / cpr;
+  if (r_in >= rpt) return;  // past the tile's last whole row: that row is the next tile's
   const int heads = static_cast<int>(nrows_total / S);
   const int row_tiles = (S + rpt - 1) / rpt;
   const int n_tiles = (heads + kRotHeads - 1) / kRotHeads * row_tiles;
@@ -138,6 +140,7 @@ __global__ void __launch_bounds__(kRotThreads) cache_write_kernel(const uint4* _
   const int cpr = D / 8;
   const int rpt = rope_rows_per_tile(D);
   const int chunk = threadIdx.x % cpr, r_in = threadIdx.x / cpr;
+  if (r_in >= rpt) return;
   const int heads = static_cast<int>(bh_count);
   const int row_tiles = (S + rpt - 1) / rpt;
   const int n_tiles = (heads + kRotHeads - 1) / kRotHeads * row_tiles;
