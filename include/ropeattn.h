@@ -165,6 +165,7 @@ RA_API ra_status rope_attn_prefill(const void* q, const void* k, const void* v, 
  * ninaddeshpande.com "Rotary positional embeddings (RoPE)".
  *   x, x_rot [B, H, S, D] bf16; x_rot may equal x (in place) but not overlap it otherwise.
  *   D even, 8 <= D <= 256 and D % 8 == 0; pos_offset >= 0. Angles are formed in fp64.
+ * Returns RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED (B * H above 2^31 - 1) or RA_ERR_CUDA.
  */
 RA_API ra_status rope_attn_rotate(const void* x, void* x_rot, int B, int H, int S, int D,
                            float rope_base, int pos_offset, ra_stream_t stream);

@@ -113,6 +113,7 @@ def test_decode_rejects(lib, kw, want):
     ((FAKE, FAKE, 1, 1, 8, 64, -1.0, 0), ra.RA_ERR_INVALID_ARG),
     ((FAKE, FAKE + 16, 1, 1, 8, 64, 1e4, 0), ra.RA_ERR_INVALID_ARG),  # partial overlap
     ((FAKE, FAKE, 1, 1, 8, 64, 1e4, -3), ra.RA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, 1 << 16, 1 << 15, 1, 8, 1e4, 0), ra.RA_ERR_UNSUPPORTED),  # 2^31 heads
 ])
 def test_rotate_rejects(lib, args, want):
     assert lib.rope_attn_rotate(*args, None) == want

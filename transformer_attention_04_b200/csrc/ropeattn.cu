@@ -1021,6 +1021,7 @@ ra_status rope_attn_rotate_rows(const void* x, void* x_rot, int B, int H, int S,
   if (x_rows < S || out_rows < S) return RA_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(B) * H * S;
   const long long heads = static_cast<long long>(B) * H;
+  if (heads > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;  // the kernel counts heads in 32 bits
   const size_t xbytes = static_cast<size_t>((heads - 1) * x_rows + S) * D * 2;
   const size_t ybytes = static_cast<size_t>((heads - 1) * out_rows + S) * D * 2;
   // in place only with the same layout; otherwise the two must not share memory
