@@ -543,9 +543,11 @@ def to_pages(Dw, cache, table):
 
 def next_rows_leg(ra, world, rank, dev, peaks):
     """The rows after the headline path, each timed on its own with CUDA events:
-    sliding-window prefill (W = 4096 over the 32k-token workload), chunked prefill into a KV
-    cache (the Llama prefill written into a cache), the decode step with in-kernel append at
-    per-sequence positions, and the same step on a paged cache (16-token pages)."""
+    sliding-window prefill (W = 4096 over the 32k-token workload); the same workload causal in
+    one call, and as a ring of 8 ranks run in turn (contiguous and zig-zag); chunked prefill
+    into a KV cache (the Llama prefill written into a cache); odd group sizes; the decode step
+    with in-kernel append at per-sequence positions, and the same step on a paged cache
+    (16-token pages)."""
     res = {}
     # sliding window: FLOPs count only the allowed pairs (4*D per pair: Q.K and P.V)
     Wl, W = LONG, WINDOW_W
@@ -557,6 +559,11 @@ def next_rows_leg(ra, world, rank, dev, peaks):
     res["sliding_window_prefill"] = _rate_entry(
         f"{Wl.name} B{Wl.B} Hq{Wl.Hq} Hkv{Wl.Hkv} S{Wl.Sq} D{Wl.D} causal, window {W}", ms, flops,
         world, "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s", "attn_fwd_sm100_kernel window")
+    # the same workload as one causal call on one GPU (the long-context configuration itself)
+    ms = time_calls(lambda: ra.rope_attn_fwd(q, k, v, Wl.rope_base, 0, True, out=out), 3)
+    res["long_context_prefill"] = _rate_entry(
+        f"{Wl.name} B{Wl.B} Hq{Wl.Hq} Hkv{Wl.Hkv} S{Wl.Sq} D{Wl.D} causal, one call", ms,
+        Wl.flops(), world, "tensor", peaks["bf16_tflops"], 1e12, "TFLOP/s")
     # ring attention: the same workload, causal, as an 8-rank ring whose ranks run in turn
     # here; per-rank times give the compute of each rank in a real ring
     ms, per_rank = ring_local_timed(ra, Wl, q, k, v, 3)
